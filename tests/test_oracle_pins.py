@@ -1,0 +1,388 @@
+"""Pins for the CPU oracle: it is checked here against things other than itself.
+
+* closed forms and special cases of the layer's definition (all-equal codes, zero scale,
+  a single expert reducing to a dense gated MLP, top-k weights summing to one);
+* an independent brute force written here in numpy float64 (own unpacking, own
+  round-to-nearest-even, no routing sort) on tiny inputs;
+* invariants: exact doubling, token permutation, routing-tensor structure;
+* an exhaustive check of the dequantisation over every code and every finite bf16 scale.
+
+The layer's definition follows the Chord blog (Novita/vLLM, German edition): subtract
+then scale in BF16 ("H200 und Blackwell indexierter Decode"), uint4 group-32 weights
+with BF16 scales ("vLLM-Integration"), block-padded sorted routing with sentinels
+("Zwei Kernel-Familien", Figure 3).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from w4a16_int4_mixture_align_b200 import inputs
+
+TOL_MAX = 2e-2   # max |a - b| <= TOL_MAX * max |b|
+TOL_MEAN = 5e-3  # sum |a - b| / sum |b| <= TOL_MEAN
+
+
+def f32(bits):
+    return oracle.bf16_to_f32(bits).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------------
+# independent helpers (float64; no code shared with oracle.c)
+
+def bf16_nearest_even(v: np.ndarray) -> np.ndarray:
+    """Nearest bf16 value to each float64 in v (values exactly representable in binary32),
+    ties to the even mantissa, overflow to +-inf: chosen between the two neighbours."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        return _bf16_nearest_even(v)
+
+
+def _bf16_nearest_even(v):
+    f = v.astype(np.float32)
+    assert np.all((f.astype(np.float64) == v) | ~np.isfinite(f))
+    bits = f.view(np.uint32)
+    lo_bits = bits & np.uint32(0xFFFF0000)
+    hi_bits = lo_bits + np.uint32(0x10000)
+    lo = lo_bits.view(np.float32).astype(np.float64)
+    hi_is_inf = (hi_bits & np.uint32(0x7FFFFFFF)) == np.uint32(0x7F800000)
+    hi = np.where(hi_is_inf, np.copysign(2.0 ** 128, v), hi_bits.view(np.float32).astype(np.float64))
+    d_lo, d_hi = np.abs(v - lo), np.abs(hi - v)
+    lo_even = ((lo_bits >> np.uint32(16)) & np.uint32(1)) == 0
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ~lo_even)
+    out = np.where(take_hi, np.where(hi_is_inf, np.copysign(np.inf, v), hi), lo)
+    return out
+
+
+def unpack_codes(qw: np.ndarray) -> np.ndarray:
+    """int32 [..., K/8] -> uint8 codes [..., K], code k%8 at bit 4*(k%8)."""
+    w = qw.view(np.uint32)
+    sh = (4 * np.arange(8, dtype=np.uint32))
+    c = (w[..., None] >> sh) & np.uint32(0xF)
+    return c.reshape(*qw.shape[:-1], qw.shape[-1] * 8).astype(np.int64)
+
+
+def dequant_f64(qw, s, rounded: bool):
+    q = unpack_codes(qw)
+    sc = np.repeat(f32(s), 32, axis=-1)
+    w = (q - 8).astype(np.float64) * sc
+    return bf16_nearest_even(w) if rounded else w
+
+
+def silu(g):
+    return g / (1.0 + np.exp(-g))
+
+
+def brute_force(d, rounded: bool):
+    """Per-token loop, no routing sort, float64 accumulation."""
+    x = f32(d["x"])
+    ids, tw = d["topk_ids"], d["topk_weights"].astype(np.float64)
+    E, N13, _ = d["qw13"].shape
+    I = N13 // 2
+    T, H = x.shape
+    out = np.zeros((T, H))
+    w13 = [dequant_f64(d["qw13"][e], d["s13"][e], rounded) for e in range(E)]
+    w2 = [dequant_f64(d["qw2"][e], d["s2"][e], rounded) for e in range(E)]
+    for t in range(T):
+        for j in range(ids.shape[1]):
+            e = ids[t, j]
+            if not (0 <= e < E):
+                continue
+            h = w13[e] @ x[t]
+            a = silu(h[:I]) * h[I:]
+            if rounded:
+                a = bf16_nearest_even(a.astype(np.float32).astype(np.float64))
+            out[t] += tw[t, j] * (w2[e] @ a)
+    return out
+
+
+def run_oracle(d, rows=None):
+    return oracle.moe_forward(d["x"], d["topk_ids"], d["topk_weights"], d["qw13"], d["s13"],
+                              d["qw2"], d["s2"], rows=rows)
+
+
+def assert_close(got_bits, ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN):
+    got = f32(got_bits)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.abs(ref).max()
+    assert scale > 0
+    err = np.abs(got - ref)
+    assert err.max() <= tol_max * scale, (err.max(), scale)
+    assert err.sum() <= tol_mean * np.abs(ref).sum(), (err.sum(), np.abs(ref).sum())
+
+
+# ----------------------------------------------------------------------------------
+# bf16 rounding and dequantisation
+
+def test_bf16_rounding_matches_nearest_even_on_random_binary32():
+    rng = np.random.default_rng(7)
+    bits = rng.integers(0, 2 ** 32, size=20000, dtype=np.uint32)
+    vals = bits.view(np.float32)
+    vals = vals[np.isfinite(vals)]
+    # include exact ties and overflow boundaries
+    ties = (np.arange(0, 4000, dtype=np.uint32) << np.uint32(16)) | np.uint32(0x8000)
+    extra = np.concatenate([ties.view(np.float32), np.float32([3.3961776e38, 3.3961775e38, -3.3961776e38, 0.0, -0.0])])
+    vals = np.concatenate([vals, extra[np.isfinite(extra)]])
+    got = f32(oracle.f32_to_bf16(vals))
+    ref = bf16_nearest_even(vals.astype(np.float64))
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), vals[~same][:5]
+
+
+def test_dequant_exhaustive_all_codes_all_finite_bf16_scales():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = (pats & 0x7F80) != 0x7F80
+    scales = pats[finite]
+    n = scales.shape[0]
+    words = np.array([0x76543210, 0xFEDCBA98, 0x76543210, 0xFEDCBA98], dtype=np.uint32)
+    qw = np.tile(words.view(np.int32), (n, 1))
+    s = scales.reshape(n, 1)
+    got = oracle.dequant(qw, s).astype(np.float64)
+    q = np.tile(np.concatenate([np.arange(16), np.arange(16)]), (n, 1))
+    exact = (q - 8) * f32(s)
+    ref = bf16_nearest_even(exact)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+    # signed zeros too: (q-8)*s == 0 only for q == 8
+    assert np.all(np.signbit(got[:, 8]) == np.signbit(f32(s)[:, 0] * 0.0))
+
+
+def test_nibble_order_low_nibble_first():
+    # word 0x89ABCDEF holds codes F,E,D,C,B,A,9,8 for k = 0..7
+    qw = np.array([[0x89ABCDEF, 0x01234567, 0, 0]], dtype=np.uint32).view(np.int32)
+    one = np.array([[0x3F80]], dtype=np.uint16)  # bf16 1.0
+    w = oracle.dequant(qw, one)[0]
+    expect = [15 - k for k in range(8)] + [7 - k for k in range(8)] + [0] * 16
+    assert list(w.astype(int)) == [c - 8 for c in expect]
+
+
+def test_group_index_is_k_over_32():
+    rng = np.random.default_rng(3)
+    qw = rng.integers(0, 2 ** 32, size=(4, 16), dtype=np.uint32).view(np.int32)  # K = 128
+    s = inputs._f32_to_bf16_bits_trunc(rng.uniform(0.5, 2.0, size=(4, 4)).astype(np.float32))
+    got = oracle.dequant(qw, s).astype(np.float64)
+    assert np.array_equal(got, dequant_f64(qw, s, rounded=True))
+
+
+# ----------------------------------------------------------------------------------
+# routing sort
+
+def brute_align(ids, E, BM):
+    T, k = ids.shape
+    n = T * k
+    flat = ids.reshape(-1)
+    cap = n + E * (BM - 1)
+    sorted_ids = [n] * cap
+    expert_ids = [-1] * ((cap + BM - 1) // BM)
+    pos = 0
+    for e in range(E):
+        mine = [f for f in range(n) if flat[f] == e]
+        start = pos
+        for r, f in enumerate(mine):
+            sorted_ids[start + r] = f
+        blocks = -(-len(mine) // BM)
+        for b in range(blocks):
+            expert_ids[start // BM + b] = e
+        pos += blocks * BM
+    return np.array(sorted_ids, np.int32), np.array(expert_ids, np.int32), pos
+
+
+@pytest.mark.parametrize("T,k,E,BM,seed", [
+    (16, 2, 8, 16, 0), (37, 8, 48, 8, 1), (5, 3, 4, 1, 2), (64, 8, 1, 16, 3),
+    (0, 8, 48, 16, 4), (100, 8, 384, 64, 5), (33, 4, 6, 256, 6), (7, 1, 3, 5, 7),
+])
+def test_align_matches_brute_force(T, k, E, BM, seed):
+    rng = np.random.default_rng(seed)
+    ids = rng.integers(-1, E + 3, size=(T, k)).astype(np.int32)  # -1 and ids >= E are not local
+    s, eids, ntp, offs = oracle.moe_align(ids, E, BM)
+    bs, beids, bntp = brute_align(ids, E, BM)
+    assert ntp == bntp
+    assert np.array_equal(s, bs)
+    assert np.array_equal(eids, beids)
+    assert offs[-1] == ntp and np.all(np.diff(offs) % BM == 0)
+
+
+def test_align_invariants_on_generated_routing():
+    cfg = inputs.CONFIGS["ep8_decode"]
+    ids, _ = inputs.make_routing(cfg)
+    BM = 8
+    s, eids, ntp, offs = oracle.moe_align(ids, cfg.E, BM)
+    n = ids.size
+    flat = ids.reshape(-1)
+    local = np.nonzero((flat >= 0) & (flat < cfg.E))[0]
+    real = s[s < n]
+    assert sorted(real.tolist()) == local.tolist()           # a permutation of local slots
+    assert ntp % BM == 0 and np.all(s[ntp:] == n)
+    for b in range(ntp // BM):                                 # one expert per block
+        blk = s[b * BM:(b + 1) * BM]
+        blk = blk[blk < n]
+        assert blk.size > 0 and np.all(flat[blk] == eids[b])
+        assert np.all(np.diff(blk) > 0)                        # increasing flat index
+    assert np.all(eids[ntp // BM:] == -1)
+
+
+def test_align_single_expert_block_one():
+    ids = np.array([[0, -1], [0, 0], [-1, 0]], dtype=np.int32)
+    s, eids, ntp, _ = oracle.moe_align(ids, 1, 1)
+    assert ntp == 4 and list(s[:4]) == [0, 2, 3, 5] and list(eids[:4]) == [0, 0, 0, 0]
+
+
+# ----------------------------------------------------------------------------------
+# the layer
+
+def tiny_inputs(seed=0, **over):
+    cfg = inputs.MoEConfig("t", over.get("T", 16), over.get("H", 256), over.get("I", 128),
+                           over.get("E", 8), over.get("E_global", over.get("E", 8)),
+                           over.get("topk", 2), over.get("routing", "normal"), seed)
+    return inputs.make_inputs(cfg)
+
+
+def test_forward_matches_brute_force_with_same_roundings():
+    d = tiny_inputs()
+    got = f32(run_oracle(d))
+    ref = brute_force(d, rounded=True)
+    # only fp32-vs-fp64 accumulation and the final bf16 rounding differ
+    assert np.abs(got - ref).max() <= 8e-3 * np.abs(ref).max()
+
+
+def test_forward_matches_exact_brute_force_within_layer_tolerance():
+    d = tiny_inputs(seed=1, T=24, E=6, topk=3)
+    assert_close(run_oracle(d), brute_force(d, rounded=False))
+
+
+def test_forward_ep_shard_with_nonlocal_slots():
+    d = tiny_inputs(seed=2, T=20, E=4, E_global=12, topk=3)
+    assert (d["topk_ids"] == -1).any()
+    got = run_oracle(d)
+    ref = brute_force(d, rounded=True)
+    no_local = ~((d["topk_ids"] >= 0).any(axis=1))
+    assert np.all(f32(got)[no_local] == 0)
+    assert np.abs(f32(got) - ref).max() <= 8e-3 * np.abs(ref).max()
+
+
+def test_subset_rows_equal_full_rows():
+    d = tiny_inputs(seed=3)
+    full = run_oracle(d)
+    rows = np.array([1, 5, 6, 15])
+    assert np.array_equal(run_oracle(d, rows=rows), full[rows])
+
+
+def test_single_expert_is_dense_gated_mlp():
+    d = tiny_inputs(seed=4, E=1, topk=1)
+    d["topk_ids"][:] = 0
+    d["topk_weights"][:] = 1.0
+    w13 = oracle.dequant(d["qw13"][0], d["s13"][0]).astype(np.float64)
+    w2 = oracle.dequant(d["qw2"][0], d["s2"][0]).astype(np.float64)
+    x = f32(d["x"])
+    h = x @ w13.T
+    I = w2.shape[1]
+    dense = (silu(h[:, :I]) * h[:, I:]) @ w2.T
+    assert_close(run_oracle(d), dense)
+
+
+def test_all_equal_codes_closed_form():
+    d = tiny_inputs(seed=5)
+    c, s_bits = 11, np.uint16(0x3C23)  # code 11, scale ~0.00995
+    word = np.uint32(sum(c << (4 * i) for i in range(8)))
+    for k in ("qw13", "qw2"):
+        d[k][:] = np.array(word).view(np.int32)
+    for k in ("s13", "s2"):
+        d[k][:] = s_bits
+    w0 = bf16_nearest_even(np.array([(c - 8) * float(f32(s_bits))]))[0]
+    x = f32(d["x"])
+    I = d["qw2"].shape[2] * 8
+    h = w0 * x.sum(axis=1)                       # every gate and up row equals this
+    a = bf16_nearest_even((silu(h) * h).astype(np.float32).astype(np.float64))
+    y = w0 * I * a                               # every output column
+    ref = np.zeros_like(x)
+    for t in range(x.shape[0]):
+        for j in range(d["topk_ids"].shape[1]):
+            if d["topk_ids"][t, j] >= 0:
+                ref[t] += d["topk_weights"][t, j] * y[t]
+    assert_close(run_oracle(d), ref, tol_max=1e-2, tol_mean=2e-3)
+
+
+def test_code_eight_gives_exact_zero():
+    d = tiny_inputs(seed=6)
+    d["qw13"][:] = np.array(np.uint32(0x88888888)).view(np.int32)
+    assert np.all(f32(run_oracle(d)) == 0)
+
+
+def test_zero_scale_gives_exact_zero():
+    d = tiny_inputs(seed=7)
+    d["s2"][:] = 0
+    assert np.all(f32(run_oracle(d)) == 0)
+
+
+def test_weights_summing_to_one_over_identical_experts_is_dense_mlp():
+    d = tiny_inputs(seed=8, topk=4)
+    for k in ("qw13", "s13", "qw2", "s2"):
+        d[k][:] = d[k][0:1]
+    w13 = oracle.dequant(d["qw13"][0], d["s13"][0]).astype(np.float64)
+    w2 = oracle.dequant(d["qw2"][0], d["s2"][0]).astype(np.float64)
+    x = f32(d["x"])
+    h = x @ w13.T
+    I = w2.shape[1]
+    dense = (silu(h[:, :I]) * h[:, I:]) @ w2.T
+    assert np.allclose(d["topk_weights"].sum(axis=1), 1.0, atol=1e-6)
+    assert_close(run_oracle(d), dense)
+
+
+def test_doubling_down_scales_doubles_output_exactly():
+    d = tiny_inputs(seed=9)
+    base = f32(run_oracle(d))
+    d["s2"] = (d["s2"].astype(np.uint32) + 0x80).astype(np.uint16)  # exponent + 1
+    assert np.array_equal(f32(run_oracle(d)), 2 * base)
+
+
+def test_doubling_topk_weights_doubles_output_exactly():
+    d = tiny_inputs(seed=10)
+    base = f32(run_oracle(d))
+    d["topk_weights"] = d["topk_weights"] * np.float32(2)
+    assert np.array_equal(f32(run_oracle(d)), 2 * base)
+
+
+def test_token_permutation_permutes_rows_bit_exactly():
+    d = tiny_inputs(seed=11)
+    base = run_oracle(d)
+    perm = np.random.default_rng(0).permutation(d["x"].shape[0])
+    for k in ("x", "topk_ids", "topk_weights"):
+        d[k] = np.ascontiguousarray(d[k][perm])
+    assert np.array_equal(run_oracle(d), base[perm])
+
+
+def test_swapped_gate_and_up_would_be_caught():
+    """A plausible mistake (gate and up halves swapped) fails the brute-force pin."""
+    d = tiny_inputs(seed=12)
+    ref = brute_force(d, rounded=True)
+    I = d["qw13"].shape[1] // 2
+    for k in ("qw13", "s13"):
+        d[k] = np.ascontiguousarray(np.concatenate([d[k][:, I:], d[k][:, :I]], axis=1))
+    wrong = f32(run_oracle(d))
+    assert np.abs(wrong - ref).max() > 0.1 * np.abs(ref).max()
+
+
+def load_golden():
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_oracle.txt")
+    g = {"out": []}
+    with open(path) as fh:
+        for line in fh:
+            if line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            if key == "out":
+                g["out"].append([int(v, 16) for v in vals[1:]])
+            else:
+                g[key] = [int(v) for v in vals]
+    g["out"] = np.array(g["out"], dtype=np.uint16)
+    return g
+
+
+def test_oracle_reproduces_golden_fixture():
+    g = load_golden()
+    d = inputs.make_inputs(inputs.CONFIGS["tiny"])
+    s, eids, ntp, offs = oracle.moe_align(d["topk_ids"], 8, 16)
+    assert ntp == g["num_tokens_padded"][0]
+    assert s.tolist() == g["sorted_ids"] and eids.tolist() == g["expert_ids"]
+    assert offs.tolist() == g["expert_offsets"]
+    assert np.array_equal(run_oracle(d), g["out"])
