@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 W4A16 mixture-of-experts layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl chord|reference]
+                    [--workload ep8_decode|ep8_prefill|tp8_decode|tp8_prefill|skew|tiny]
+
+One step = one layer call through the C ABI: routing sort (chord_moe_align) then
+chord_moe_forward (gate_up GEMM + SiLU*up, down GEMM + top-k weight, combine), on a
+synthetic Kimi-K2-shaped batch already resident in HBM. The default workload is the
+EP8 decode shard: 128 tokens, hidden 7168, moe_intermediate 2048, experts 0..47 of
+384 local, top-8 from uniform router logits. Weights (1.19 GB) exceed the 126 MB L2,
+so no flush is needed between steps.
+
+Prints one JSON line (rank 0). `value` is microseconds per layer call for the whole job:
+the max over ranks of the timed region divided by (steps x ranks), since each rank runs
+an independent replica (the layer does not shard across GPUs here).
+
+--impl reference times the CPU oracle (test infrastructure) on the same workload on
+the host cores: rank 0 only, other ranks exit without work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a16_int4_mixture_align_b200 import inputs  # noqa: E402
+
+METRIC = "W4A16 MoE layer µs/call; decode eff. HBM GB/s, prefill TFLOPS vs roofline"
+UNIT = "us/call"
+GATE_UP_BYTES_PER_EXPERT = None  # computed from the config
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+DEFAULT_STEPS = {"ep8_decode": 2000, "tp8_decode": 2000, "tiny": 2000, "ep8_prefill": 200,
+                 "tp8_prefill": 400, "skew": 100}
+
+
+def describe(cfg: inputs.MoEConfig) -> str:
+    shard = f"experts 0..{cfg.E - 1} of {cfg.E_global} local" if cfg.E < cfg.E_global else f"all {cfg.E} experts"
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} I={cfg.I} {shard} top-{cfg.topk} "
+            f"{cfg.routing} router logits, int4 group-32 bf16 scales")
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def algorithmic_work(cfg: inputs.MoEConfig, ids: np.ndarray):
+    """Bytes and FLOPs a layer call must move/compute, from the routing alone."""
+    E, H, I = cfg.E, cfg.H, cfg.I
+    flat = ids.reshape(-1)
+    local = flat[(flat >= 0) & (flat < E)]
+    R = int(local.size)
+    active = int(np.unique(local).size)
+    gu_w = 2 * I * H // 2 + 2 * I * (H // 32) * 2        # codes + scales of one expert
+    dn_w = H * I // 2 + H * (I // 32) * 2
+    tokens_local = int(((ids >= 0) & (ids < E)).any(axis=1).sum())
+    gate_up = {"weights": active * gu_w, "x": tokens_local * H * 2, "a": R * I * 2}
+    down = {"weights": active * dn_w, "a": R * I * 2, "y": R * H * 4}
+    combine = {"y": R * H * 4, "out": cfg.T * H * 2}
+    return {
+        "R": R, "active_experts": active,
+        "gate_up_bytes": sum(gate_up.values()), "down_bytes": sum(down.values()),
+        "combine_bytes": sum(combine.values()),
+        "layer_bytes": active * (gu_w + dn_w) + cfg.T * H * 2 * 2,
+        "gate_up_flops": 2 * R * H * 2 * I, "down_flops": 2 * R * I * H,
+        "unit_gate_up_bytes": gu_w,
+    }
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU works."""
+
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sms, maxes, reasons, n = [], [], set(), 0
+        for ts, line in self.lines:
+            if ts < t0 - 0.2 or ts > t1 + 0.2:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            n += 1
+            try:
+                sms.append(float(parts[2]))
+                maxes.append(float(parts[3]))
+            except ValueError:
+                pass
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sms) if sms else None,
+                "sm_max_mhz": max(maxes) if maxes else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ------------------------------------------------------------------------------ chord arm
+
+def src_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)[kernel_key][workload]
+    except Exception:
+        return None
+    if rec.get("src_sha") != src_digest(rec["sources"]):
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+def run_chord(args, rank, world, local_rank):
+    import torch
+    from w4a16_int4_mixture_align_b200 import chord
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = inputs.CONFIGS[args.workload]
+    weights = inputs.make_weights(cfg)
+    rcfg = inputs.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})  # each replica its own batch
+    ids_np, tw_np = inputs.make_routing(rcfg)
+    x_np = inputs.make_hidden(rcfg)
+    work = algorithmic_work(cfg, ids_np)
+
+    layer = chord.ChordMoE(weights[0], weights[1].view(np.int16), weights[2], weights[3].view(np.int16),
+                           topk=cfg.topk, E_global=cfg.E_global, max_tokens=cfg.T, device=dev)
+    del weights
+    x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    ids = torch.from_numpy(ids_np).to(dev)
+    tw = torch.from_numpy(tw_np).to(dev)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, ids, tw, out=out)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    assert layer.check_status() == 0
+
+    # per-kernel events: [start, align done, gate_up done, down done, combine done] per step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = chord.chord_launch_count()
+    t_wall0 = time.time()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        layer.align(ids)
+        chord.chord_set_timing_events(ev[k][1:5])
+        chord.chord_moe_forward(x, ids, tw, layer.sorted_ids, layer.expert_ids, layer.ntp, layer.block_m,
+                                layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace)
+        chord.chord_set_timing_events(None)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    launches = chord.chord_launch_count() - launches0
+    elapsed_ms = start.elapsed_time(stop)
+    assert layer.check_status() == 0
+
+    seg = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in range(K)])
+    seg_ms = seg.mean(axis=0)  # align, gate_up, down, combine
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
+    ids_h = torch.from_numpy(ids_np).pin_memory()
+    tw_h = torch.from_numpy(tw_np).pin_memory()
+    out_h = torch.empty((cfg.T, cfg.H), dtype=torch.int16).pin_memory()
+    xd, idsd, twd = torch.empty_like(x), torch.empty_like(ids), torch.empty_like(tw)
+
+    def e2e_step():
+        xd.view(torch.int16).copy_(x_h, non_blocking=True)
+        idsd.copy_(ids_h, non_blocking=True)
+        twd.copy_(tw_h, non_blocking=True)
+        layer.forward(xd, idsd, twd, out=out)
+        out_h.copy_(out.view(torch.int16), non_blocking=True)
+
+    for _ in range(W):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler.stop()
+    e2e_ms = s2.elapsed_time(e2)
+    h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    # ---- max over ranks
+    stats = torch.tensor([elapsed_ms, e2e_ms, *seg_ms.tolist()], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(stats[0]), float(stats[1])
+    seg_ms = stats[2:].cpu().numpy()
+    if rank != 0:
+        return None
+
+    hbm, tf_burst, tf_sust, pk_kind = peaks()
+    us_call = elapsed_ms * 1000.0 / (K * world)
+    gu_us, dn_us = seg_ms[1] * 1000.0, seg_ms[2] * 1000.0
+    decode = layer.block_m <= 32
+    if decode:
+        achieved = work["gate_up_bytes"] / (gu_us * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "kernel": "stream_gemm gate_up", "achieved": round(achieved, 1),
+                    "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                    "peak_source": f"{pk_kind} hbm_gbs",
+                    "traffic": recorded_traffic("stream_gemm_gate_up", args.workload),
+                    "algorithmic_bytes_per_launch": work["gate_up_bytes"]}
+    else:
+        achieved = work["gate_up_flops"] / (gu_us * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": "gate_up GEMM", "achieved": round(achieved, 1),
+                    "peak": tf_burst, "unit": "TFLOP/s", "frac": round(achieved / tf_burst, 4),
+                    "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                    "traffic": recorded_traffic("tc_gemm_gate_up", args.workload),
+                    "algorithmic_flops_per_launch": work["gate_up_flops"]}
+    layer_us = elapsed_ms * 1000.0 / K
+    line = {
+        "metric": METRIC, "value": round(us_call, 3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(elapsed_ms / K, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "block_m": layer.block_m,
+                   "schedule": "weight-streaming" if decode else "tensor-core",
+                   "routed_pairs": work["R"], "active_experts": work["active_experts"],
+                   "l2": "no flush: weights %.2f GB > 126 MB L2" % (work["layer_bytes"] / 1e9),
+                   "parallelism": f"replicas x{world}"},
+        "kernels_us": {"align": round(seg_ms[0] * 1000, 2), "gate_up": round(gu_us, 2),
+                       "down": round(dn_us, 2), "combine": round(seg_ms[3] * 1000, 2),
+                       "gate_up+down": round(gu_us + dn_us, 2)},
+        "layer": {"GB/s": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9, 1),
+                  "hbm_frac": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9 / hbm, 4),
+                  "TFLOP/s": round((work["gate_up_flops"] + work["down_flops"]) / (layer_us * 1e-6) / 1e12, 2)},
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_ms * 1000.0 / (K * world), 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    return line
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------ oracle arms
+
+def oracle_call(d, threads):
+    import oracle
+    return oracle.moe_forward(d["x"], d["topk_ids"], d["topk_weights"], d["qw13"], d["s13"],
+                              d["qw2"], d["s2"], n_threads=threads)
+
+
+def cpu_baseline(cfg, max_seconds=30.0):
+    """The oracle as it stands on the host cores: full layer calls, repeated while the
+    total stays within ~max_seconds (at least one call)."""
+    import oracle
+    oracle.build()
+    d = inputs.make_inputs(cfg)
+    threads = os.cpu_count() or 1
+    times = []
+    t_total = time.time()
+    while True:
+        t0 = time.time()
+        oracle_call(d, threads)
+        times.append(time.time() - t0)
+        if time.time() - t_total + times[-1] > max_seconds or len(times) >= 5:
+            break
+    us = statistics.median(times) * 1e6
+    return {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{len(times)} full layer call(s) of the workload (all {cfg.T} tokens), median"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    cfg = inputs.CONFIGS[args.workload]
+    d = inputs.make_inputs(cfg)
+    threads = os.cpu_count() or 1
+    for _ in range(args.warmup):
+        oracle_call(d, threads)
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle_call(d, threads)
+    el = time.time() - t0
+    us = el * 1e6 / args.steps
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1000 / args.steps, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": describe(cfg), "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"each step one full layer call of the workload (all {cfg.T} tokens)"},
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["chord", "reference"], default="chord")
+    ap.add_argument("--workload", choices=list(inputs.CONFIGS), default="ep8_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 3 if args.impl == "reference" else DEFAULT_STEPS[args.workload]
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the oracle runs on rank 0 alone; other ranks exit without work
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    line = run_chord(args, rank, world, local_rank)
+    if line is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inputs.CONFIGS[args.workload])
+        else:
+            line["cpu_baseline"] = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

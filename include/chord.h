@@ -1,0 +1,197 @@
+/*
+ * chord.h -- C ABI of the B200 (sm_100a) W4A16 mixture-of-experts layer.
+ *
+ * The layer (Novita/vLLM blog "vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel fuer
+ * Kimi K2.x"; sections cited below by their headings) takes BF16 activations, uint4
+ * weights packed eight per int32 along K, and one BF16 scale per 32 consecutive K
+ * elements of each output row ("vLLM-Integration": uint4, group-32, BF16 scales). A
+ * weight element is w = bf16((q - 8) * s), subtract first, then scale, rounded once to
+ * BF16 ("H200 und Blackwell indexierter Decode").
+ *
+ *   out[t] = sum over local top-k slots j of  topk_weights[t,j] * W2[e] . act(W13[e] . x[t])
+ *   act(h) = silu(h[0:I]) * h[I:2I]      (rounded to BF16 before the down projection)
+ *
+ * with FP32 accumulation throughout (F16 accumulation is not offered; "vLLM-Integration",
+ * deployment notes).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument named as "device" is a CUDA device pointer owned by the
+ *    caller. The library allocates no device or host memory on any call.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL means the legacy default
+ *    stream) and returns before it runs. No entry point reads device memory back to
+ *    the host, so align + forward can be captured in a CUDA graph ("vLLM-Integration":
+ *    the indexed fast path consumes over-allocated routing buffers without reading the
+ *    routed count back to the host).
+ *  - Argument errors are detected on the host before anything is enqueued and returned
+ *    as a chord_status_t; chord_last_error_detail() then describes the failure (the
+ *    text is thread-local and valid until the next call on the same thread).
+ *  - Errors found on the device (routing validation, weight-blob header mismatch, a
+ *    bounded wait that gave up) are OR-ed into a status word inside the forward
+ *    workspace and read with chord_moe_check_status().
+ *  - Device code is built for sm_100a only. On any other device the entry points that
+ *    launch work return CHORD_ERR_UNSUPPORTED.
+ */
+#ifndef CHORD_H_
+#define CHORD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CHORD_API __attribute__((visibility("default")))
+#else
+#define CHORD_API
+#endif
+
+typedef struct CUstream_st* chord_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  CHORD_OK = 0,
+  CHORD_ERR_INVALID_ARG = 1,        /* null pointer, negative or inconsistent size */
+  CHORD_ERR_UNSUPPORTED = 2,        /* group size != 32, unsupported shape, not sm_100 */
+  CHORD_ERR_LAYOUT_MISMATCH = 3,    /* weight blob of another role/shape/layout */
+  CHORD_ERR_WORKSPACE_TOO_SMALL = 4,
+  CHORD_ERR_CUDA = 5,               /* a CUDA runtime call failed (see detail text) */
+  CHORD_ERR_DEVICE = 6              /* chord_moe_check_status found device status bits */
+} chord_status_t;
+
+/* Device status bits (chord_moe_check_status). */
+#define CHORD_DEV_ROUTING_INVALID 0x1u /* VALIDATE_ROUTING found inconsistent routing */
+#define CHORD_DEV_BLOB_MISMATCH   0x2u /* a weight blob header does not match the call */
+#define CHORD_DEV_TIMEOUT         0x4u /* a bounded on-chip wait gave up */
+
+/* Weight roles for chord_repack_weights. */
+#define CHORD_ROLE_GATE_UP 1 /* W13 [E, 2I, H]: rows [0,I) gate, rows [I,2I) up */
+#define CHORD_ROLE_DOWN    2 /* W2  [E, H, I] */
+
+/* Flags for chord_moe_forward. */
+#define CHORD_FLAG_VALIDATE_ROUTING 0x1 /* check routing tensors on the device first */
+#define CHORD_FLAG_FORCE_STREAM     0x2 /* force the weight-streaming (decode) schedule */
+#define CHORD_FLAG_FORCE_TENSOR     0x4 /* force the tensor-core (prefill) schedule */
+
+CHORD_API const char* chord_status_string(int status);
+CHORD_API const char* chord_last_error_detail(void);
+
+/* ------------------------------------------------------------------------------------
+ * Routing sort ("Zwei Kernel-Familien": the indexed family consumes vLLM's
+ * sorted_ids / expert_ids / num_tokens_padded; Figure 3: activations stay unpadded and
+ * the routing indices carry padding sentinels).
+ *
+ * Flat slot index f = t*topk + j. A slot is local when 0 <= topk_ids[f] < E; any other
+ * id (-1, or a global id of an expert on another shard) is skipped. With c_e the local
+ * slots of expert e, p_e = ceil(c_e / block_m) * block_m and off_e = sum_{e' < e} p_e':
+ *   sorted_ids[off_e + r] = the r-th local flat index of expert e, in increasing f;
+ *   every other entry of sorted_ids (up to the capacity below) = T*topk (sentinel);
+ *   expert_ids[b] = e for the p_e / block_m blocks of expert e, in increasing e, and
+ *   -1 for every block at or past num_tokens_padded / block_m;
+ *   num_tokens_padded[0] = off_E;   expert_offsets[e] = off_e for e in [0, E].
+ * An expert with no local slot gets no block. The result is deterministic.
+ *
+ * Capacities: sorted_ids holds chord_moe_align_capacity() int32, expert_ids holds
+ * chord_moe_align_num_blocks() int32. Limits: 1 <= E <= 1024, 1 <= block_m <= 256,
+ * capacity < 2^31. `workspace` (device, >= chord_moe_align_workspace_bytes() bytes,
+ * any content, 256-byte aligned) is scratch for large T*topk; it may be NULL when
+ * that size is 0. expert_offsets (device, E+1 int32) may be NULL.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API int64_t chord_moe_align_capacity(int64_t T, int topk, int E, int block_m);
+CHORD_API int64_t chord_moe_align_num_blocks(int64_t T, int topk, int E, int block_m);
+CHORD_API size_t chord_moe_align_workspace_bytes(int64_t T, int topk, int E);
+CHORD_API chord_status_t chord_moe_align(const int32_t* topk_ids /* device [T, topk] */, int64_t T,
+                               int topk, int E, int block_m, int32_t* sorted_ids,
+                               int32_t* expert_ids, int32_t* num_tokens_padded /* [1] */,
+                               int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
+                               size_t workspace_bytes, chord_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * One-time weight repack ("Gruppierte SM90-Kernel": prepared weights are permuted INT4
+ * buffers with re-laid scales, and the mode is recorded in the prepared weight and
+ * checked at dispatch; Figure 2: layouts are fixed at model load).
+ *
+ * In:  qweight (device) int32 [E, N, K/8]: code of (n, k) in bits 4*(k%8)..+3 of word
+ *      [n, k/8] (low nibble first); scales (device) bf16 bits [E, N, K/32].
+ *      For CHORD_ROLE_GATE_UP, N = 2*I with gate rows first; for CHORD_ROLE_DOWN, N = H.
+ * Out: `out` (device, >= chord_repacked_bytes() bytes, 256-byte aligned): an opaque
+ *      blob = 256-byte header (magic, version, role, E, N, K, group) + codes + scales
+ *      in the tile layout the forward kernels read (128 rows x 128 K per tile; gate and
+ *      up rows interleaved in blocks of 8 for CHORD_ROLE_GATE_UP).
+ * Requires group_size == 32 (else CHORD_ERR_UNSUPPORTED), N % 128 == 0, K % 128 == 0.
+ * The input buffers may be freed once the stream has run the repack.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API size_t chord_repacked_bytes(int E, int N, int K, int group_size);
+CHORD_API chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scales, int E,
+                                    int N, int K, int group_size, int role, void* out,
+                                    size_t out_bytes, chord_stream_t stream);
+
+/* Inverse layout, for checks: blob -> logical-order bf16 weights w[E, N, K] computed
+ * with the forward kernels' own dequantisation (rows in the caller's logical order).
+ * w_bf16: device, E*N*K uint16. */
+CHORD_API chord_status_t chord_dequant_weights(const void* blob, size_t blob_bytes, uint16_t* w_bf16,
+                                     chord_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Schedule selector ("Kernel-Optimierungen": the tokens routed per expert, tok_e, not
+ * the total token count, decide the schedule; below ~80 tokens per expert the indexed
+ * resolver keeps a block-count search, above it sizes block_m around each expert's
+ * padded rows). Host-only and memoised. Returns the block_m to pass to
+ * chord_moe_align and chord_moe_forward. Small values (<= 32) select the
+ * weight-streaming schedule in chord_moe_forward, larger ones the tensor-core
+ * schedule. tok_e is estimated without reading routing back: T*topk / E_global.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API int chord_select_block_m(int64_t T, int topk, int E_local, int E_global, int H, int I);
+
+/* ------------------------------------------------------------------------------------
+ * The layer.
+ *
+ * hidden       device bf16 [T, H]
+ * topk_ids     device int32 [T, topk] (same convention as chord_moe_align)
+ * topk_weights device fp32  [T, topk]; not renormalised over local slots
+ * sorted_ids, expert_ids, num_tokens_padded: device routing tensors for this block_m
+ *              (from chord_moe_align or any producer with the same contract; entries
+ *              >= T*topk are padding, blocks with expert_ids outside [0,E) are skipped)
+ * w13, w2      device blobs from chord_repack_weights (roles GATE_UP [E,2I,H], DOWN [E,H,I])
+ * out          device bf16 [T, H]; every row is written (0 for tokens with no local slot)
+ * workspace    device, >= chord_moe_workspace_bytes(), 256-byte aligned. Its first 256
+ *              bytes hold the device status word: zero them once after allocating; the
+ *              rest is scratch that needs no initialisation.
+ *
+ * Requires H % 128 == 0, I % 128 == 0, 1 <= block_m <= 256 (same as used for align).
+ * Concurrent forwards must not share a workspace.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API size_t chord_moe_workspace_bytes(int64_t T, int topk, int E, int H, int I, int block_m);
+CHORD_API chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids,
+                                 const float* topk_weights, const int32_t* sorted_ids,
+                                 const int32_t* expert_ids, const int32_t* num_tokens_padded,
+                                 int block_m, const void* w13, const void* w2, int64_t T,
+                                 int H, int I, int E, int topk, uint16_t* out, void* workspace,
+                                 size_t workspace_bytes, int flags, chord_stream_t stream);
+
+/* Synchronises `stream`, copies the workspace status word to *device_status, clears it
+ * on the device, and returns CHORD_OK when it was zero, else CHORD_ERR_DEVICE. */
+CHORD_API chord_status_t chord_moe_check_status(void* workspace, chord_stream_t stream,
+                                      uint32_t* device_status);
+
+/* ------------------------------------------------------------------------------------
+ * Measurement hooks (no counterpart on the pages; used by the benchmark).
+ *
+ * chord_set_timing_events: while set (n == 4), every chord_moe_forward made on the
+ * calling thread records the caller-owned cudaEvent_t handles events[0..3] on its
+ * stream: [0] before the first GEMM, [1] between the gate_up and down GEMMs, [2] after
+ * the down GEMM, [3] after the combine. n == 0 clears the hook. The handles must stay
+ * valid while set. Returns CHORD_ERR_INVALID_ARG for other n or null handles.
+ *
+ * chord_launch_count: number of CUDA kernels this library has launched in the process
+ * (all entry points, all threads), for checking launch counts of a timed region.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API chord_status_t chord_set_timing_events(void* const* events, int n);
+CHORD_API uint64_t chord_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CHORD_H_ */

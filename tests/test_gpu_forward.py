@@ -1,0 +1,212 @@
+"""The whole layer on the GPU vs the CPU oracle.
+
+Tiny workload: every output element. Kimi-K2-shaped workloads at full size: a seeded
+sample of 512 token rows among those with a local slot (all such rows when fewer),
+computed one by one by the oracle, in the same launch configuration the benchmark
+times. Both schedules (weight streaming and tensor core) are checked where they apply.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import assert_layer_close, bf16_bits_to_f64, ensure_built
+from w4a16_int4_mixture_align_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def chord():
+    ensure_built()
+    from w4a16_int4_mixture_align_b200 import chord as c
+    return c
+
+
+def to_dev(d):
+    import torch
+    dev = torch.device("cuda")
+    return {
+        "x": torch.from_numpy(d["x"].view(np.int16)).to(dev).view(torch.bfloat16),
+        "ids": torch.from_numpy(d["topk_ids"]).to(dev),
+        "w": torch.from_numpy(d["topk_weights"]).to(dev),
+    }
+
+
+def make_layer(chord, d, block_m=None, max_tokens=None):
+    cfg = d["cfg"]
+    return chord.ChordMoE(d["qw13"], d["s13"].view(np.int16), d["qw2"], d["s2"].view(np.int16),
+                          topk=cfg.topk, E_global=cfg.E_global,
+                          max_tokens=max_tokens or cfg.T, block_m=block_m)
+
+
+def run_layer(layer, d, flags=0):
+    import torch
+    t = to_dev(d)
+    out = layer(t["x"], t["ids"], t["w"], flags=flags)
+    torch.cuda.synchronize()
+    st = layer.check_status()
+    assert st == 0, hex(st)
+    return out.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def oracle_rows(d, rows):
+    return oracle.moe_forward(d["x"], d["topk_ids"], d["topk_weights"], d["qw13"], d["s13"],
+                              d["qw2"], d["s2"], rows=rows)
+
+
+# ------------------------------------------------------------------------------ tiny
+
+@pytest.fixture(scope="module")
+def tiny():
+    return inputs.make_inputs(inputs.CONFIGS["tiny"])
+
+
+@pytest.mark.parametrize("block_m", [1, 8, 16, 32, 64, 256])
+@pytest.mark.parametrize("path", ["stream", "tensor"])
+def test_tiny_full_output(chord, tiny, block_m, path):
+    flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR
+    layer = make_layer(chord, tiny, block_m=block_m)
+    got = run_layer(layer, tiny, flags)
+    ref = oracle_rows(tiny, None)
+    assert_layer_close(got, ref)
+
+
+def test_tiny_matches_golden_fixture_within_tolerance(chord, tiny):
+    import os
+    g = {}
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.txt")
+    rows = []
+    for line in open(path):
+        if line.startswith("out "):
+            rows.append([int(v, 16) for v in line.split()[2:]])
+    ref = np.array(rows, dtype=np.uint16)
+    got = run_layer(make_layer(chord, tiny), tiny)
+    assert_layer_close(got, ref)
+
+
+# ------------------------------------------------------------------------------ full size
+
+BIG = ["ep8_decode", "ep8_prefill", "tp8_decode", "tp8_prefill", "skew"]
+
+
+@pytest.fixture(scope="module")
+def big_inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cache.clear()
+            cache[name] = inputs.make_inputs(inputs.CONFIGS[name])
+        return cache[name]
+    return get
+
+
+@pytest.mark.parametrize("name", BIG)
+def test_full_size_sampled_rows(chord, big_inputs, name):
+    d = big_inputs(name)
+    cfg = d["cfg"]
+    layer = make_layer(chord, d)
+    got = run_layer(layer, d)
+    rows = inputs.sample_rows(d["topk_ids"], cfg.E, 512, seed=1)
+    ref = oracle_rows(d, rows)
+    r = assert_layer_close(got[rows], ref)
+    # rows without a local slot are exactly zero
+    none = ~((d["topk_ids"] >= 0) & (d["topk_ids"] < cfg.E)).any(axis=1)
+    assert np.all(bf16_bits_to_f64(got[none]) == 0)
+    print(name, "block_m", layer.block_m, r)
+
+
+# ------------------------------------------------------------------------------ edges
+
+def small_inputs(T, E=8, E_global=None, topk=2, H=256, I=128, seed=3):
+    cfg = inputs.MoEConfig("edge", T, H, I, E, E_global or E, topk, "normal", seed)
+    return inputs.make_inputs(cfg)
+
+
+@pytest.mark.parametrize("T", [1, 3, 37, 129])
+@pytest.mark.parametrize("path", ["stream", "tensor"])
+def test_ragged_token_counts(chord, T, path):
+    d = small_inputs(T, E=6, E_global=10, topk=3, H=384, I=256)
+    flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR
+    got = run_layer(make_layer(chord, d, block_m=16), d, flags)
+    assert_layer_close(got, oracle_rows(d, None))
+
+
+@pytest.mark.parametrize("path", ["stream", "tensor"])
+def test_no_local_slot_gives_zero_rows(chord, path):
+    d = small_inputs(20)
+    d["topk_ids"][:] = -1
+    flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR
+    got = run_layer(make_layer(chord, d, block_m=8), d, flags)
+    assert np.all(bf16_bits_to_f64(got) == 0)
+
+
+def test_single_expert_topk1(chord):
+    d = small_inputs(33, E=1, topk=1)
+    got = run_layer(make_layer(chord, d, block_m=8), d)
+    assert_layer_close(got, oracle_rows(d, None))
+
+
+def test_one_expert_takes_everything(chord):
+    d = small_inputs(300, E=4, topk=2)
+    d["topk_ids"][:, 0] = 2
+    d["topk_ids"][:, 1] = -1
+    for bm in (8, 256):
+        got = run_layer(make_layer(chord, d, block_m=bm), d)
+        assert_layer_close(got, oracle_rows(d, None))
+
+
+def test_repeated_calls_are_deterministic_in_routing_and_stable(chord, tiny):
+    layer = make_layer(chord, tiny, block_m=8)
+    a = run_layer(layer, tiny)
+    b = run_layer(layer, tiny)
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------------------ errors
+
+def test_swapped_weight_roles_fail_on_host(chord, tiny):
+    import torch
+    layer = make_layer(chord, tiny, block_m=8)
+    t = to_dev(tiny)
+    layer.align(t["ids"])
+    out = torch.empty((16, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(chord.ChordError) as ei:
+        chord.chord_moe_forward(t["x"], t["ids"], t["w"], layer.sorted_ids, layer.expert_ids, layer.ntp,
+                                layer.block_m, layer.w2, layer.w13, layer.I, layer.E, out, layer.workspace)
+    assert ei.value.status == chord.CHORD_ERR_LAYOUT_MISMATCH
+
+
+def test_foreign_blob_header_checked_on_device(chord, tiny):
+    import torch
+    layer = make_layer(chord, tiny, block_m=8)
+    t = to_dev(tiny)
+    layer.align(t["ids"])
+    # copies the host registry does not know: the kernels check the header themselves
+    w13c, w2c = layer.w2.clone(), layer.w13.clone()          # roles swapped
+    out = torch.zeros((16, 256), dtype=torch.bfloat16, device="cuda")
+    chord.chord_moe_forward(t["x"], t["ids"], t["w"], layer.sorted_ids, layer.expert_ids, layer.ntp,
+                            layer.block_m, w13c, w2c, layer.I, layer.E, out, layer.workspace,
+                            chord.CHORD_FLAG_FORCE_STREAM)
+    st = layer.check_status()
+    assert st & chord.CHORD_DEV_BLOB_MISMATCH
+    assert layer.check_status() == 0  # cleared by the read
+
+
+def test_routing_validation_flags_corrupt_tensors(chord, tiny):
+    import torch
+    layer = make_layer(chord, tiny, block_m=8)
+    t = to_dev(tiny)
+    layer.align(t["ids"])
+    out = torch.zeros((16, 256), dtype=torch.bfloat16, device="cuda")
+    bad = layer.expert_ids.clone()
+    bad[0] = 1000
+    chord.chord_moe_forward(t["x"], t["ids"], t["w"], layer.sorted_ids, bad, layer.ntp,
+                            layer.block_m, layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace,
+                            chord.CHORD_FLAG_VALIDATE_ROUTING | chord.CHORD_FLAG_FORCE_STREAM)
+    assert layer.check_status() & chord.CHORD_DEV_ROUTING_INVALID
+    # valid routing passes validation
+    chord.chord_moe_forward(t["x"], t["ids"], t["w"], layer.sorted_ids, layer.expert_ids, layer.ntp,
+                            layer.block_m, layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace,
+                            chord.CHORD_FLAG_VALIDATE_ROUTING)
+    assert layer.check_status() == 0

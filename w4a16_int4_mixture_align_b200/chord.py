@@ -1,0 +1,264 @@
+"""Python binding of libchord.so (include/chord.h): argument marshalling only.
+
+Every function keeps its C name and forwards torch CUDA tensors as raw device pointers
+on the current torch stream. Nothing here computes any part of the layer; when the
+library is missing the import fails loudly (there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libchord.so")
+
+CHORD_OK = 0
+CHORD_ERR_INVALID_ARG = 1
+CHORD_ERR_UNSUPPORTED = 2
+CHORD_ERR_LAYOUT_MISMATCH = 3
+CHORD_ERR_WORKSPACE_TOO_SMALL = 4
+CHORD_ERR_CUDA = 5
+CHORD_ERR_DEVICE = 6
+
+CHORD_DEV_ROUTING_INVALID = 0x1
+CHORD_DEV_BLOB_MISMATCH = 0x2
+CHORD_DEV_TIMEOUT = 0x4
+
+CHORD_ROLE_GATE_UP = 1
+CHORD_ROLE_DOWN = 2
+
+CHORD_FLAG_VALIDATE_ROUTING = 0x1
+CHORD_FLAG_FORCE_STREAM = 0x2
+CHORD_FLAG_FORCE_TENSOR = 0x4
+
+# every symbol include/chord.h declares: (name, restype, argtypes)
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "chord_status_string": (ctypes.c_char_p, [_I]),
+    "chord_last_error_detail": (ctypes.c_char_p, []),
+    "chord_moe_align_capacity": (_I64, [_I64, _I, _I, _I]),
+    "chord_moe_align_num_blocks": (_I64, [_I64, _I, _I, _I]),
+    "chord_moe_align_workspace_bytes": (_SZ, [_I64, _I, _I]),
+    "chord_moe_align": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "chord_repacked_bytes": (_SZ, [_I, _I, _I, _I]),
+    "chord_repack_weights": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "chord_dequant_weights": (_I, [_P, _SZ, _P, _P]),
+    "chord_select_block_m": (_I, [_I64, _I, _I, _I, _I, _I]),
+    "chord_moe_workspace_bytes": (_SZ, [_I64, _I, _I, _I, _I, _I]),
+    "chord_moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _I64, _I, _I, _I, _I, _P, _P,
+                               _SZ, _I, _P]),
+    "chord_moe_check_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
+    "chord_launch_count": (ctypes.c_uint64, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run `python -m w4a16_int4_mixture_align_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+class ChordError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        detail = lib().chord_last_error_detail().decode()
+        name = lib().chord_status_string(status).decode()
+        super().__init__(f"{what}: {name}: {detail}")
+        self.status = status
+
+
+def _check(status: int, what: str):
+    if status != CHORD_OK:
+        raise ChordError(status, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "device tensors must be contiguous CUDA tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+# --------------------------------------------------------------------------- sizes
+
+def chord_moe_align_capacity(T, topk, E, block_m) -> int:
+    return int(lib().chord_moe_align_capacity(T, topk, E, block_m))
+
+
+def chord_moe_align_num_blocks(T, topk, E, block_m) -> int:
+    return int(lib().chord_moe_align_num_blocks(T, topk, E, block_m))
+
+
+def chord_moe_align_workspace_bytes(T, topk, E) -> int:
+    return int(lib().chord_moe_align_workspace_bytes(T, topk, E))
+
+
+def chord_repacked_bytes(E, N, K, group_size=32) -> int:
+    return int(lib().chord_repacked_bytes(E, N, K, group_size))
+
+
+def chord_select_block_m(T, topk, E_local, E_global, H, I) -> int:
+    return int(lib().chord_select_block_m(T, topk, E_local, E_global, H, I))
+
+
+def chord_moe_workspace_bytes(T, topk, E, H, I, block_m) -> int:
+    return int(lib().chord_moe_workspace_bytes(T, topk, E, H, I, block_m))
+
+
+def chord_status_string(status: int) -> str:
+    return lib().chord_status_string(status).decode()
+
+
+def chord_last_error_detail() -> str:
+    return lib().chord_last_error_detail().decode()
+
+
+# --------------------------------------------------------------------------- calls
+
+def chord_moe_align(topk_ids, E, block_m, sorted_ids, expert_ids, num_tokens_padded,
+                    expert_offsets=None, workspace=None, stream=None):
+    T, topk = topk_ids.shape
+    ws_bytes = 0 if workspace is None else _nbytes(workspace)
+    _check(lib().chord_moe_align(_ptr(topk_ids), T, topk, E, block_m, _ptr(sorted_ids),
+                                 _ptr(expert_ids), _ptr(num_tokens_padded), _ptr(expert_offsets),
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "chord_moe_align")
+
+
+def chord_repack_weights(qweight, scales, role, out, group_size=32, stream=None):
+    E, N, K8 = qweight.shape
+    _check(lib().chord_repack_weights(_ptr(qweight), _ptr(scales), E, N, K8 * 8, group_size, role,
+                                      _ptr(out), _nbytes(out), _stream(stream)),
+           "chord_repack_weights")
+
+
+def chord_dequant_weights(blob, w_out, stream=None):
+    _check(lib().chord_dequant_weights(_ptr(blob), _nbytes(blob), _ptr(w_out), _stream(stream)),
+           "chord_dequant_weights")
+
+
+def chord_moe_forward(hidden, topk_ids, topk_weights, sorted_ids, expert_ids, num_tokens_padded,
+                      block_m, w13, w2, I, E, out, workspace, flags=0, stream=None):
+    T, H = hidden.shape
+    topk = topk_ids.shape[1]
+    _check(lib().chord_moe_forward(_ptr(hidden), _ptr(topk_ids), _ptr(topk_weights),
+                                   _ptr(sorted_ids), _ptr(expert_ids), _ptr(num_tokens_padded),
+                                   block_m, _ptr(w13), _ptr(w2), T, H, I, E, topk, _ptr(out),
+                                   _ptr(workspace), _nbytes(workspace), flags, _stream(stream)),
+           "chord_moe_forward")
+
+
+def chord_moe_check_status(workspace, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    st = lib().chord_moe_check_status(_ptr(workspace), _stream(stream), ctypes.byref(v))
+    if st not in (CHORD_OK, CHORD_ERR_DEVICE):
+        _check(st, "chord_moe_check_status")
+    return int(v.value)
+
+
+def chord_set_timing_events(events=None):
+    """events: four torch.cuda.Event (already recorded once, so their handles exist) or None."""
+    if not events:
+        _check(lib().chord_set_timing_events(None, 0), "chord_set_timing_events")
+        return
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().chord_set_timing_events(arr, 4), "chord_set_timing_events")
+
+
+def chord_launch_count() -> int:
+    return int(lib().chord_launch_count())
+
+
+# --------------------------------------------------------------------------- convenience
+
+def _alloc_bytes(n: int, device) -> torch.Tensor:
+    # 256-byte alignment: the torch caching allocator returns 512-byte aligned blocks
+    t = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    assert t.data_ptr() % 256 == 0
+    return t
+
+
+class ChordMoE:
+    """A prepared layer: repacked weights plus reusable routing and workspace buffers.
+
+    Buffers are sized for up to ``max_tokens`` tokens; call with any T <= max_tokens.
+    ``block_m`` defaults to the library's selector for ``max_tokens``.
+    """
+
+    def __init__(self, qw13, s13, qw2, s2, topk, E_global=None, max_tokens=1, block_m=None,
+                 device="cuda"):
+        E, N13, H8 = qw13.shape
+        self.E, self.I, self.H, self.topk = E, N13 // 2, H8 * 8, topk
+        self.E_global = E if E_global is None else E_global
+        self.device = torch.device(device)
+        self.w13 = _alloc_bytes(chord_repacked_bytes(E, N13, self.H), self.device)
+        self.w2 = _alloc_bytes(chord_repacked_bytes(E, self.H, self.I), self.device)
+        dev = lambda a: torch.as_tensor(a).to(self.device).contiguous()  # noqa: E731
+        chord_repack_weights(dev(qw13), dev(s13), CHORD_ROLE_GATE_UP, self.w13)
+        chord_repack_weights(dev(qw2), dev(s2), CHORD_ROLE_DOWN, self.w2)
+        torch.cuda.current_stream().synchronize()
+        self.max_tokens = 0
+        self.block_m = block_m
+        self.reserve(max_tokens)
+
+    def reserve(self, T: int, block_m=None):
+        if block_m is not None:
+            self.block_m = block_m
+        elif self.block_m is None:
+            self.block_m = chord_select_block_m(T, self.topk, self.E, self.E_global, self.H, self.I)
+        bm = self.block_m
+        cap = chord_moe_align_capacity(T, self.topk, self.E, bm)
+        nb = chord_moe_align_num_blocks(T, self.topk, self.E, bm)
+        d = self.device
+        self.sorted_ids = torch.empty(max(cap, 1), dtype=torch.int32, device=d)
+        self.expert_ids = torch.empty(max(nb, 1), dtype=torch.int32, device=d)
+        self.ntp = torch.zeros(1, dtype=torch.int32, device=d)
+        self.offsets = torch.empty(self.E + 1, dtype=torch.int32, device=d)
+        aw = chord_moe_align_workspace_bytes(T, self.topk, self.E)
+        self.align_ws = _alloc_bytes(aw, d) if aw else None
+        self.workspace = torch.zeros(chord_moe_workspace_bytes(T, self.topk, self.E, self.H, self.I, bm),
+                                     dtype=torch.uint8, device=d)
+        self.max_tokens = T
+
+    def align(self, topk_ids):
+        chord_moe_align(topk_ids, self.E, self.block_m, self.sorted_ids, self.expert_ids, self.ntp,
+                        self.offsets, self.align_ws)
+
+    def forward(self, hidden, topk_ids, topk_weights, out=None, flags=0):
+        T = hidden.shape[0]
+        if T > self.max_tokens:
+            self.reserve(T)
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        self.align(topk_ids)
+        chord_moe_forward(hidden, topk_ids, topk_weights, self.sorted_ids, self.expert_ids, self.ntp,
+                          self.block_m, self.w13, self.w2, self.I, self.E, out, self.workspace, flags)
+        return out
+
+    __call__ = forward
+
+    def check_status(self) -> int:
+        return chord_moe_check_status(self.workspace)

@@ -1,0 +1,350 @@
+// api.cu -- the C ABI declared in include/chord.h: argument checks, the prepared-weight
+// registry, the memoised schedule selector and the launch sequence of the layer.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <unordered_map>
+
+#include "chord_internal.cuh"
+
+namespace chord {
+namespace {
+
+thread_local char g_detail[512] = "";
+thread_local cudaEvent_t g_timing[4] = {nullptr, nullptr, nullptr, nullptr};
+thread_local bool g_timing_on = false;
+std::atomic<uint64_t> g_launches{0};
+
+chord_status_t fail(chord_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+chord_status_t cuda_fail(cudaError_t err, const char* what) {
+  return fail(CHORD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+struct DeviceInfo {
+  bool ok = false;
+  int num_sms = 0;
+  int major = 0, minor = 0;
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceInfo> g_devices;
+
+struct BlobInfo {
+  int E, N, K, role;
+  size_t bytes;
+};
+std::unordered_map<const void*, BlobInfo> g_blobs;
+std::map<std::tuple<int64_t, int, int, int, int, int>, int> g_select_cache;
+
+chord_status_t current_device(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_devices.find(dev);
+  if (it == g_devices.end()) {
+    DeviceInfo d;
+    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    d.ok = (d.major == 10 && d.minor == 0);
+    it = g_devices.emplace(dev, d).first;
+  }
+  *out = it->second;
+  if (!out->ok)
+    return fail(CHORD_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                dev, out->major, out->minor);
+  return CHORD_OK;
+}
+
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+chord_status_t check_align_args(int64_t T, int topk, int E, int block_m) {
+  if (T < 0 || topk < 1 || topk > 64)
+    return fail(CHORD_ERR_INVALID_ARG, "T=%lld topk=%d", (long long)T, topk);
+  if (E < 1 || E > 1024) return fail(CHORD_ERR_UNSUPPORTED, "E=%d outside [1, 1024]", E);
+  if (block_m < 1 || block_m > 256)
+    return fail(CHORD_ERR_UNSUPPORTED, "block_m=%d outside [1, 256]", block_m);
+  const int64_t cap = T * topk + int64_t(E) * (block_m - 1);
+  if (cap >= (int64_t(1) << 31)) return fail(CHORD_ERR_UNSUPPORTED, "routing capacity %lld >= 2^31", (long long)cap);
+  return CHORD_OK;
+}
+
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+
+}  // namespace chord
+
+using namespace chord;
+
+extern "C" {
+
+const char* chord_status_string(int status) {
+  switch (status) {
+    case CHORD_OK: return "CHORD_OK";
+    case CHORD_ERR_INVALID_ARG: return "CHORD_ERR_INVALID_ARG";
+    case CHORD_ERR_UNSUPPORTED: return "CHORD_ERR_UNSUPPORTED";
+    case CHORD_ERR_LAYOUT_MISMATCH: return "CHORD_ERR_LAYOUT_MISMATCH";
+    case CHORD_ERR_WORKSPACE_TOO_SMALL: return "CHORD_ERR_WORKSPACE_TOO_SMALL";
+    case CHORD_ERR_CUDA: return "CHORD_ERR_CUDA";
+    case CHORD_ERR_DEVICE: return "CHORD_ERR_DEVICE";
+    default: return "CHORD_ERR_UNKNOWN";
+  }
+}
+
+const char* chord_last_error_detail(void) { return g_detail; }
+
+int64_t chord_moe_align_capacity(int64_t T, int topk, int E, int block_m) {
+  if (T < 0 || topk < 1 || E < 1 || block_m < 1) return -1;
+  return T * topk + int64_t(E) * (block_m - 1);
+}
+
+int64_t chord_moe_align_num_blocks(int64_t T, int topk, int E, int block_m) {
+  const int64_t cap = chord_moe_align_capacity(T, topk, E, block_m);
+  if (cap < 0) return -1;
+  return (cap + block_m - 1) / block_m;
+}
+
+size_t chord_moe_align_workspace_bytes(int64_t T, int topk, int E) {
+  if (T < 0 || topk < 1 || E < 1) return 0;
+  return align_workspace_bytes(T * topk, E);
+}
+
+chord_status_t chord_moe_align(const int32_t* topk_ids, int64_t T, int topk, int E, int block_m,
+                               int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_tokens_padded,
+                               int32_t* expert_offsets, void* workspace, size_t workspace_bytes,
+                               chord_stream_t stream) {
+  g_detail[0] = 0;
+  chord_status_t st = check_align_args(T, topk, E, block_m);
+  if (st != CHORD_OK) return st;
+  if ((T > 0 && !topk_ids) || !sorted_ids || !expert_ids || !num_tokens_padded)
+    return fail(CHORD_ERR_INVALID_ARG, "null routing pointer");
+  const size_t need = align_workspace_bytes(T * topk, E);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "align workspace needs %zu bytes, got %zu", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (need > 0 && !aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  const int64_t cap = chord_moe_align_capacity(T, topk, E, block_m);
+  const int64_t nblocks = chord_moe_align_num_blocks(T, topk, E, block_m);
+  cudaError_t err = launch_align(topk_ids, T * topk, E, block_m, cap, nblocks, sorted_ids,
+                                 expert_ids, num_tokens_padded, expert_offsets, workspace,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_align launch");
+  return CHORD_OK;
+}
+
+size_t chord_repacked_bytes(int E, int N, int K, int group_size) {
+  if (E < 1 || N < 1 || K < 1 || group_size != kGroup || N % kTileN || K % kTileK) return 0;
+  return size_t(blob_total_bytes(E, N, K));
+}
+
+chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scales, int E, int N,
+                                    int K, int group_size, int role, void* out, size_t out_bytes,
+                                    chord_stream_t stream) {
+  g_detail[0] = 0;
+  if (group_size != kGroup)
+    return fail(CHORD_ERR_UNSUPPORTED, "group_size=%d; only group-32 scales are supported", group_size);
+  if (role != CHORD_ROLE_GATE_UP && role != CHORD_ROLE_DOWN)
+    return fail(CHORD_ERR_INVALID_ARG, "role=%d", role);
+  if (E < 1 || N < 1 || K < 1) return fail(CHORD_ERR_INVALID_ARG, "E=%d N=%d K=%d", E, N, K);
+  if (N % kTileN || K % kTileK)
+    return fail(CHORD_ERR_UNSUPPORTED, "N=%d and K=%d must be multiples of 128", N, K);
+  if (!qweight || !scales || !out) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if (!aligned256(out)) return fail(CHORD_ERR_INVALID_ARG, "output blob not 256-byte aligned");
+  const size_t need = size_t(blob_total_bytes(E, N, K));
+  if (out_bytes < need) return fail(CHORD_ERR_INVALID_ARG, "blob needs %zu bytes, got %zu", need, out_bytes);
+  chord_status_t st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  cudaError_t err = launch_repack(qweight, scales, E, N, K, role, static_cast<uint8_t*>(out),
+                                  reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "repack launch");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_blobs[out] = BlobInfo{E, N, K, role, need};
+  return CHORD_OK;
+}
+
+chord_status_t chord_dequant_weights(const void* blob, size_t blob_bytes, uint16_t* w_bf16,
+                                     chord_stream_t stream) {
+  g_detail[0] = 0;
+  if (!blob || !w_bf16) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  BlobInfo info;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_blobs.find(blob);
+    if (it == g_blobs.end())
+      return fail(CHORD_ERR_LAYOUT_MISMATCH, "blob was not prepared by chord_repack_weights in this process");
+    info = it->second;
+  }
+  if (blob_bytes < info.bytes) return fail(CHORD_ERR_INVALID_ARG, "blob_bytes too small");
+  chord_status_t st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  cudaError_t err = launch_dequant_blob(static_cast<const uint8_t*>(blob), info.E, info.N, info.K,
+                                        info.role, w_bf16, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "dequant launch");
+  return CHORD_OK;
+}
+
+int chord_select_block_m(int64_t T, int topk, int E_local, int E_global, int H, int I) {
+  if (T < 0 || topk < 1 || E_local < 1 || E_global < E_local) return -1;
+  const auto key = std::make_tuple(T, topk, E_local, E_global, H, I);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_select_cache.find(key);
+    if (it != g_select_cache.end()) return it->second;
+  }
+  // expected routed tokens per local expert, without reading the routing back
+  const double tok_e = double(T) * topk / double(E_global);
+  int bm;
+  if (tok_e <= 4.0) bm = 8;
+  else if (tok_e <= 10.0) bm = 16;
+  else if (tok_e <= 24.0) bm = 32;
+  else bm = 256;  // tensor-core schedule: one block per expert (up to 256 rows)
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_select_cache[key] = bm;
+  return bm;
+}
+
+size_t chord_moe_workspace_bytes(int64_t T, int topk, int E, int H, int I, int block_m) {
+  if (T < 0 || topk < 1 || E < 1 || H < 1 || I < 1 || block_m < 1) return 0;
+  return size_t(forward_workspace(T, topk, E, H, I, block_m).total);
+}
+
+chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids,
+                                 const float* topk_weights, const int32_t* sorted_ids,
+                                 const int32_t* expert_ids, const int32_t* num_tokens_padded,
+                                 int block_m, const void* w13, const void* w2, int64_t T, int H,
+                                 int I, int E, int topk, uint16_t* out, void* workspace,
+                                 size_t workspace_bytes, int flags, chord_stream_t stream_) {
+  g_detail[0] = 0;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  chord_status_t st = check_align_args(T, topk, E, block_m);
+  if (st != CHORD_OK) return st;
+  if (H < kTileK || H % kTileK || I < kTileK || I % kTileK)
+    return fail(CHORD_ERR_UNSUPPORTED, "H=%d and I=%d must be positive multiples of 128", H, I);
+  if ((flags & CHORD_FLAG_FORCE_STREAM) && (flags & CHORD_FLAG_FORCE_TENSOR))
+    return fail(CHORD_ERR_INVALID_ARG, "FORCE_STREAM and FORCE_TENSOR are exclusive");
+  if (!w13 || !w2 || !workspace || !sorted_ids || !expert_ids || !num_tokens_padded)
+    return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if (T > 0 && (!hidden || !topk_ids || !topk_weights || !out))
+    return fail(CHORD_ERR_INVALID_ARG, "null activation pointer");
+  if (!aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(CHORD_ERR_INVALID_ARG, "hidden and out must be 16-byte aligned");
+  const ForwardWorkspace ws = forward_workspace(T, topk, E, H, I, block_m);
+  if (workspace_bytes < ws.total)
+    return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "forward workspace needs %llu bytes, got %zu",
+                (unsigned long long)ws.total, workspace_bytes);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto check = [&](const void* p, int role, int N, int K, const char* name) -> chord_status_t {
+      auto it = g_blobs.find(p);
+      if (it == g_blobs.end()) return CHORD_OK;  // foreign blob: the kernels check its header
+      const BlobInfo& b = it->second;
+      if (b.role != role || b.E != E || b.N != N || b.K != K)
+        return fail(CHORD_ERR_LAYOUT_MISMATCH,
+                    "%s blob is role %d [E=%d N=%d K=%d], call needs role %d [E=%d N=%d K=%d]", name,
+                    b.role, b.E, b.N, b.K, role, E, N, K);
+      return CHORD_OK;
+    };
+    if ((st = check(w13, CHORD_ROLE_GATE_UP, 2 * I, H, "w13")) != CHORD_OK) return st;
+    if ((st = check(w2, CHORD_ROLE_DOWN, H, I, "w2")) != CHORD_OK) return st;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if (T == 0) return CHORD_OK;
+
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  ForwardArgs a{};
+  a.x = hidden;
+  a.topk_ids = topk_ids;
+  a.topk_weights = topk_weights;
+  a.sorted_ids = sorted_ids;
+  a.expert_ids = expert_ids;
+  a.ntp = num_tokens_padded;
+  a.w13 = static_cast<const uint8_t*>(w13);
+  a.w2 = static_cast<const uint8_t*>(w2);
+  a.out = out;
+  a.a = reinterpret_cast<uint16_t*>(wsb + ws.a_offset);
+  a.y = reinterpret_cast<float*>(wsb + ws.y_offset);
+  a.status = reinterpret_cast<uint32_t*>(wsb);
+  a.T = T;
+  a.H = H;
+  a.I = I;
+  a.E = E;
+  a.topk = topk;
+  a.block_m = block_m;
+  a.cap = chord_moe_align_capacity(T, topk, E, block_m);
+  a.num_sms = dev.num_sms;
+
+  cudaError_t err;
+  if (flags & CHORD_FLAG_VALIDATE_ROUTING) {
+    if ((err = launch_validate(a, stream)) != cudaSuccess) return cuda_fail(err, "validate launch");
+  }
+  const bool timing = g_timing_on;
+  if (timing && (err = cudaEventRecord(g_timing[0], stream)) != cudaSuccess)
+    return cuda_fail(err, "timing event");
+  const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) ||
+                      (!(flags & CHORD_FLAG_FORCE_STREAM) && block_m > 32);
+  cudaEvent_t mid = timing ? g_timing[1] : nullptr;
+  err = tensor ? launch_tc_gemms(a, stream, mid) : launch_stream_gemms(a, stream, mid);
+  if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");
+  if (timing && (err = cudaEventRecord(g_timing[2], stream)) != cudaSuccess)
+    return cuda_fail(err, "timing event");
+  if ((err = launch_combine(a, stream)) != cudaSuccess) return cuda_fail(err, "combine launch");
+  if (timing && (err = cudaEventRecord(g_timing[3], stream)) != cudaSuccess)
+    return cuda_fail(err, "timing event");
+  return CHORD_OK;
+}
+
+chord_status_t chord_set_timing_events(void* const* events, int n) {
+  g_detail[0] = 0;
+  if (n == 0) {
+    g_timing_on = false;
+    return CHORD_OK;
+  }
+  if (n != 4 || !events) return fail(CHORD_ERR_INVALID_ARG, "need exactly 4 events, got %d", n);
+  for (int i = 0; i < 4; ++i) {
+    if (!events[i]) return fail(CHORD_ERR_INVALID_ARG, "null event %d", i);
+    g_timing[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_timing_on = true;
+  return CHORD_OK;
+}
+
+uint64_t chord_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+chord_status_t chord_moe_check_status(void* workspace, chord_stream_t stream_, uint32_t* device_status) {
+  g_detail[0] = 0;
+  if (!workspace) return fail(CHORD_ERR_INVALID_ARG, "null workspace");
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  uint32_t v = 0;
+  cudaError_t err = cudaStreamSynchronize(stream);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaStreamSynchronize");
+  err = cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess) return cuda_fail(err, "status read");
+  if (v != 0) {
+    err = cudaMemsetAsync(workspace, 0, sizeof v, stream);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(stream);
+    if (err != cudaSuccess) return cuda_fail(err, "status clear");
+  }
+  if (device_status) *device_status = v;
+  if (v != 0) return fail(CHORD_ERR_DEVICE, "device status 0x%x", v);
+  return CHORD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,299 @@
+// chord_internal.cuh -- shared definitions of the sm_100a W4A16 MoE kernels.
+//
+// Repacked weight blob (written by chord_repack_weights, read by the GEMM kernels):
+//
+//   [0, 256)        BlobHeader
+//   codes           E * N * K / 2 bytes, 256-byte aligned
+//   scales          E * N * (K/32) * 2 bytes, 256-byte aligned
+//
+// Codes are grouped in tiles of 128 physical rows x 128 K (8 KiB), tile (e, nt, kt)
+// at byte ((e * N/128 + nt) * K/128 + kt) * 8192. A tile is 8 sub-tiles of 16 rows
+// (rb = 0..7, 1 KiB each). Inside a sub-tile the int32 word index is
+//     h*128 + g*16 + t*4 + j         (h 0..1, g 0..7, t 0..3, j 0..3)
+// and holds physical row  rb*16 + 8h + g  and K range  kt*128 + 32j + 8t + [0, 8).
+// Lane (g, t) of a warp therefore reads its two 16-byte vectors (h = 0, 1) from
+// contiguous 512-byte spans. Inside a word, K offset u (0..7) sits in nibble
+// (u >> 1) + 4 * (u & 1), so that masking nibbles {i, i+4} after a right shift by 4i
+// yields the bf16 pair (u = 2i, 2i+1) in order.
+//
+// Scales are tiled the same way: 1 KiB per tile, 128 bytes per sub-tile, bf16 index
+//     g*8 + h*4 + j      for physical row rb*16 + 8h + g, group kt*4 + j.
+//
+// Physical row p maps to a logical row: for the down projection p itself; for gate_up
+// (N = 2I) block p/16 holds gate rows 8*(p/16) + [0, 8) followed by the matching up
+// rows I + 8*(p/16) + [0, 8), so a tile carries the gate and up halves of the same
+// intermediate columns for the fused SiLU*up epilogue.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/chord.h"
+
+namespace chord {
+
+constexpr uint32_t kBlobMagic = 0x34574843u;  // "CHW4"
+constexpr uint32_t kBlobVersion = 1;
+constexpr uint32_t kLayoutTile128 = 1;
+constexpr int kGroup = 32;
+constexpr int kTileN = 128;
+constexpr int kTileK = 128;
+constexpr int kTileCodeBytes = kTileN * kTileK / 2;          // 8192
+constexpr int kTileScaleBytes = kTileN * (kTileK / kGroup) * 2;  // 1024
+constexpr int kHeaderBytes = 256;
+
+struct BlobHeader {
+  uint32_t magic;
+  uint32_t version;
+  uint32_t layout;
+  uint32_t role;
+  int32_t E, N, K, group;
+  uint64_t codes_offset;
+  uint64_t scales_offset;
+  uint64_t total_bytes;
+  uint32_t reserved[50];
+};
+static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
+
+__host__ __device__ inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+__host__ __device__ inline uint64_t blob_codes_bytes(int E, int N, int K) {
+  return uint64_t(E) * N * (K / 2);
+}
+__host__ __device__ inline uint64_t blob_scales_bytes(int E, int N, int K) {
+  return uint64_t(E) * N * (K / kGroup) * 2;
+}
+__host__ __device__ inline uint64_t blob_codes_offset() { return kHeaderBytes; }
+__host__ __device__ inline uint64_t blob_scales_offset(int E, int N, int K) {
+  return align256(kHeaderBytes + blob_codes_bytes(E, N, K));
+}
+__host__ __device__ inline uint64_t blob_total_bytes(int E, int N, int K) {
+  return align256(blob_scales_offset(E, N, K) + blob_scales_bytes(E, N, K));
+}
+
+// Logical row of physical row p in a tile-layout matrix with N physical rows.
+__host__ __device__ inline int logical_row(int role, int N, int p) {
+  if (role != CHORD_ROLE_GATE_UP) return p;
+  int blk = p >> 4, r = p & 15;
+  return r < 8 ? (blk * 8 + r) : (N / 2 + blk * 8 + (r - 8));
+}
+
+// Nibble slot holding K offset u (0..7) of a repacked word.
+__host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1); }
+
+// ------------------------------------------------------------------------------------
+// Workspace of chord_moe_forward: [status 256 B][a: cap x I bf16][y: T*topk x H fp32]
+struct ForwardWorkspace {
+  uint64_t a_offset, y_offset, total;
+};
+__host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int topk, int E, int H,
+                                                              int I, int block_m) {
+  ForwardWorkspace w;
+  int64_t cap = T * topk + int64_t(E) * (block_m - 1);
+  w.a_offset = 256;
+  w.y_offset = align256(w.a_offset + uint64_t(cap) * I * 2);
+  w.total = align256(w.y_offset + uint64_t(T) * topk * H * 4);
+  return w;
+}
+
+// ------------------------------------------------------------------------------------
+// PTX helpers (sm_100a)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Any on-chip wait gives up after this long, flags CHORD_DEV_TIMEOUT and unwinds.
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of `bar` to complete. Returns false (and raises the CTA's
+// abort flag and the device status) when the wait gave up or another thread aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, CHORD_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// One bulk copy global -> shared, completing `bytes` of transaction on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (createpolicy result).
+__device__ __forceinline__ void bulk_g2s_hint(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// ------------------------------------------------------------------------------------
+// int4 -> bf16 dequantisation, subtract first, then scale, each rounded in BF16.
+//
+// 0x4300 | q is the bf16 bit pattern of 128 + q (q < 16 fills mantissa bits 0..3), so
+// subtracting 136 gives q - 8 exactly; the product with the bf16 scale is rounded once
+// (round-to-nearest-even), matching bf16((q - 8) * s).
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(bits));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// word: one repacked int32 (eight codes); s2: the group scale in both halves.
+// out[i] = bf16 pair for K offsets (2i, 2i+1) of the word's 8-element run.
+__device__ __forceinline__ void dequant8(uint32_t word, uint32_t s2, uint32_t out[4]) {
+  const uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u, k136 = 0x43084308u;
+  out[0] = bf16x2_mul(bf16x2_sub(lop3_and_or(word, kMask, kMagic), k136), s2);
+  out[1] = bf16x2_mul(bf16x2_sub(lop3_and_or(word >> 4, kMask, kMagic), k136), s2);
+  out[2] = bf16x2_mul(bf16x2_sub(lop3_and_or(word >> 8, kMask, kMagic), k136), s2);
+  out[3] = bf16x2_mul(bf16x2_sub(lop3_and_or(word >> 12, kMask, kMagic), k136), s2);
+}
+
+__device__ __forceinline__ uint32_t bf16_splat(uint16_t s) { return uint32_t(s) * 0x10001u; }
+
+// D (f32 16x8) += A (bf16 16x16, row) * B (bf16 16x8, col). Not volatile: a pure
+// function of its operands, so the compiler may interleave it with independent work.
+__device__ __forceinline__ void mma_bf16_16816(float c[4], const uint32_t a[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return g / (1.0f + __expf(-g)) * u;
+}
+
+// ------------------------------------------------------------------------------------
+// Kernel launchers (defined in the .cu files; return cudaGetLastError()).
+
+cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int64_t cap,
+                         int64_t nblocks, int32_t* sorted_ids, int32_t* expert_ids,
+                         int32_t* ntp, int32_t* offsets, void* workspace, cudaStream_t stream);
+size_t align_workspace_bytes(int64_t n, int E);
+
+cudaError_t launch_repack(const int32_t* qweight, const uint16_t* scales, int E, int N, int K,
+                          int role, uint8_t* blob, cudaStream_t stream);
+cudaError_t launch_dequant_blob(const uint8_t* blob, int E, int N, int K, int role,
+                                uint16_t* w, cudaStream_t stream);
+
+struct ForwardArgs {
+  const uint16_t* x;
+  const int32_t* topk_ids;
+  const float* topk_weights;
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntp;
+  const uint8_t* w13;
+  const uint8_t* w2;
+  uint16_t* out;
+  uint16_t* a;     // [cap, I] bf16 intermediate, indexed by sorted position
+  float* y;        // [T*topk, H] fp32 weighted expert outputs, indexed by flat slot
+  uint32_t* status;
+  int64_t T;
+  int H, I, E, topk, block_m;
+  int64_t cap;     // sorted_ids capacity
+  int num_sms;
+};
+
+// Adds n to the process-wide kernel launch counter (chord_launch_count).
+void count_launches(int n);
+
+// `mid` (may be null) is recorded on the stream between the gate_up and down GEMMs.
+cudaError_t launch_validate(const ForwardArgs& a, cudaStream_t stream);
+cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid);
+cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid);
+cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream);
+
+}  // namespace chord

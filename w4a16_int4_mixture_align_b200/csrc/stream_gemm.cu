@@ -1,0 +1,396 @@
+// stream_gemm.cu -- weight-streaming W4A16 grouped GEMMs (few routed tokens per expert).
+//
+// With few tokens routed to each expert the layer is bound by reading the packed
+// weights once from HBM. The Chord blog's decode profile swaps the MMA operands so the
+// dequantised weights fill the MMA-M slot and uses m16n8k16 ("H200 und Blackwell
+// indexierter Decode"); the same operand orientation is used here, on sm_100a, with the
+// weight tiles streamed by bulk asynchronous copies through a deep shared-memory ring:
+//
+//   warp 0        producer: per item (routing block b, token chunk c, 128-row tile nt)
+//                 it publishes a descriptor, then per 128-wide K step issues one 8 KiB
+//                 code copy, one 1 KiB scale copy and one 256-byte copy per routed
+//                 activation row, all completing on the stage's mbarrier.
+//   warps 1..8    consumer group 0, warps 9..16 group 1: group g takes the K steps of
+//                 parity g; warp w owns 16 physical rows. Codes go shared -> registers,
+//                 dequantise to bf16 pairs (subtract 8, then scale) that are exactly the
+//                 A fragments of mma.m16n8k16; tokens are the N dimension.
+//   epilogue      group 1 hands its partial sums to group 0, which adds them and applies
+//                 SiLU(gate)*up (gate_up; gate and up rows are interleaved by the repack)
+//                 or the top-k weight (down, written to the per-slot buffer y).
+//
+// Every wait is an mbarrier wait bounded in time; on timeout the CTA raises
+// CHORD_DEV_TIMEOUT, unwinds, and the producer waits (bounded) for its copies in flight.
+#include "chord_internal.cuh"
+
+namespace chord {
+namespace {
+
+constexpr int kConsumerWarps = 16;          // two groups of 8
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kActPitch = 320;              // bytes per activation row in a stage (256 + 64 pad)
+constexpr int kDescRing = 32;
+constexpr int kMaxTC = 32;
+
+enum Epi { kGateUp = 0, kDown = 1 };
+
+struct StreamParams {
+  const uint32_t* codes;    // blob codes region
+  const uint16_t* scales;   // blob scales region
+  const uint8_t* blob;      // header
+  int N, K;                 // physical rows, reduction length
+  int E, role;
+  const uint16_t* act;      // gate_up: x [T, H]; down: a [cap, I]
+  int act_ld;               // elements per activation row (H or I)
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntp;
+  int block_m;
+  int64_t n_slots;          // T * topk
+  int topk;
+  int64_t cap;
+  uint16_t* a_out;          // gate_up output [cap, I]
+  float* y_out;             // down output [T*topk, H]
+  const float* topk_weights;
+  int I, H;
+  uint32_t* status;
+};
+
+struct ItemDesc {
+  int e, nt, pos0, end;     // end = 1 marks the end of the item sequence
+  int f[kMaxTC];            // flat slot of each token column, -1 when padding
+};
+
+template <int TC>
+struct Smem {
+  static constexpr int kStageCodes = 0;
+  static constexpr int kStageScales = kTileCodeBytes;
+  static constexpr int kStageAct = kTileCodeBytes + kTileScaleBytes;
+  static constexpr int kStageBytes = ((kStageAct + TC * kActPitch) + 127) / 128 * 128;
+  static constexpr int kHandoverBytes = 8 * 32 * (TC / 8) * 4 * 4;  // 8 warps x 32 lanes x 4*NT floats
+  static constexpr int kBudget = 200 * 1024;
+  static constexpr int kFit =
+      (kBudget - kHandoverBytes - kDescRing * int(sizeof(ItemDesc)) - 1024) / kStageBytes;
+  static constexpr int kStages = kFit > 24 ? 24 : kFit;
+  static constexpr int kBytes =
+      kStages * kStageBytes + kHandoverBytes + kDescRing * int(sizeof(ItemDesc)) + 1024;
+};
+
+template <int EPI, int TC>
+__global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p) {
+  using S = Smem<TC>;
+  constexpr int NT8 = TC / 8;
+  constexpr int NSTAGE = S::kStages;
+  static_assert(NSTAGE >= 4 && NSTAGE < kDescRing, "stage count");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* stages = smem;
+  float* handover = reinterpret_cast<float*>(smem + NSTAGE * S::kStageBytes);
+  ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + NSTAGE * S::kStageBytes + S::kHandoverBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(descs) +
+                                               kDescRing * sizeof(ItemDesc));
+  uint64_t* full = bars;                        // [NSTAGE]
+  uint64_t* empty = full + NSTAGE;              // [NSTAGE]
+  uint64_t* dfull = empty + NSTAGE;             // [kDescRing]
+  uint64_t* dempty = dfull + kDescRing;         // [kDescRing]
+  uint64_t* hfull = dempty + kDescRing;         // [1] group 1 -> group 0
+  uint64_t* hempty = hfull + 1;                 // [1] group 0 -> group 1
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    const BlobHeader* hd = reinterpret_cast<const BlobHeader*>(p.blob);
+    if (hd->magic != kBlobMagic || hd->version != kBlobVersion || hd->layout != kLayoutTile128 ||
+        int(hd->role) != p.role || hd->E != p.E || hd->N != p.N || hd->K != p.K) {
+      abort_flag = 2;
+      if (blockIdx.x == 0) atomicOr(p.status, CHORD_DEV_BLOB_MISMATCH);
+    }
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);
+    }
+    for (int s = 0; s < kDescRing; ++s) {
+      mbar_init(&dfull[s], 1);
+      mbar_init(&dempty[s], 8);
+    }
+    mbar_init(hfull, 8);
+    mbar_init(hempty, 8);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (abort_flag) return;
+  volatile int* abort_v = &abort_flag;
+
+  const int KT = p.K / kTileK;
+  const int NTILES = p.N / kTileN;
+  const int cpb = (p.block_m + TC - 1) / TC;  // token chunks per routing block
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    int ntp = *p.ntp;
+    if (ntp < 0) ntp = 0;
+    if (ntp > p.cap) ntp = int(p.cap);
+    const int64_t nblocks = ntp / p.block_m;
+    const int64_t items = nblocks * cpb * NTILES;
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_a = policy_evict_last();
+    uint32_t stage = 0;      // global stage counter
+    uint32_t nitem = 0;      // published descriptors
+    for (int64_t w = blockIdx.x;; w += gridDim.x) {
+      const bool end = w >= items;
+      int e = -1, nt = 0, pos0 = 0, fval = -1;
+      if (!end) {
+        nt = int(w % NTILES);
+        const int64_t bc = w / NTILES;
+        const int64_t b = bc / cpb;
+        const int c = int(bc % cpb);
+        e = __ldg(p.expert_ids + b);
+        pos0 = int(b * p.block_m) + c * TC;
+        const int lim = int(b * p.block_m) + p.block_m;
+        if (lane < TC && pos0 + lane < lim) {
+          const int f = __ldg(p.sorted_ids + pos0 + lane);
+          if (f >= 0 && f < p.n_slots) fval = f;
+        }
+        if (unsigned(e) >= unsigned(p.E)) fval = -1;
+        if (__ballot_sync(0xffffffffu, fval >= 0) == 0) continue;  // nothing routed here
+      }
+      // publish the item (or the end marker) to the consumers
+      const uint32_t ds = nitem % kDescRing;
+      if (nitem >= kDescRing &&
+          !mbar_wait(&dempty[ds], ((nitem / kDescRing) - 1) & 1, abort_v, p.status))
+        break;
+      ItemDesc* d = &descs[ds];
+      if (lane < TC) d->f[lane] = fval;
+      if (lane == 0) {
+        d->e = e; d->nt = nt; d->pos0 = pos0; d->end = end ? 1 : 0;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dfull[ds]);
+      ++nitem;
+      if (end) break;
+      // stream the item's K steps
+      const unsigned rows = __ballot_sync(0xffffffffu, fval >= 0);
+      const uint32_t bytes = kTileCodeBytes + kTileScaleBytes + __popc(rows) * 256u;
+      const int64_t act_row = (EPI == kGateUp) ? int64_t(fval / p.topk) : int64_t(pos0 + lane);
+      const uint16_t* act_src = p.act + act_row * p.act_ld;
+      const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt, ++stage) {
+        const uint32_t slot = stage % NSTAGE;
+        if (stage >= uint32_t(NSTAGE) &&
+            !mbar_wait(&empty[slot], ((stage / NSTAGE) - 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = stages + slot * S::kStageBytes;
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+        __syncwarp();
+        if (lane == 0) {
+          bulk_g2s_hint(st + S::kStageCodes,
+                        reinterpret_cast<const uint8_t*>(p.codes) + (tile0 + kt) * kTileCodeBytes,
+                        kTileCodeBytes, &full[slot], pol_w);
+          bulk_g2s_hint(st + S::kStageScales,
+                        reinterpret_cast<const uint8_t*>(p.scales) + (tile0 + kt) * kTileScaleBytes,
+                        kTileScaleBytes, &full[slot], pol_w);
+        }
+        if (fval >= 0)
+          bulk_g2s_hint(st + S::kStageAct + lane * kActPitch, act_src + kt * kTileK, 256,
+                        &full[slot], pol_a);
+      }
+      if (!ok) break;
+    }
+    // drain: wait (bounded, ignoring the abort flag) for every copy still in flight
+    if (lane == 0) {
+      int dummy = 0;
+      const uint32_t first = stage > uint32_t(NSTAGE) ? stage - NSTAGE : 0;
+      for (uint32_t s = first; s < stage; ++s)
+        mbar_wait(&full[s % NSTAGE], (s / NSTAGE) & 1, &dummy, p.status);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int cw = warp - 1;             // 0..15
+  const int grp = cw >> 3;             // 0 or 1
+  const int rb = cw & 7;               // 16-row block inside the tile
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t stage0 = 0;                 // stage counter at the item's first K step
+  for (uint32_t it = 0;; ++it) {
+    const uint32_t ds = it % kDescRing;
+    if (!mbar_wait(&dfull[ds], (it / kDescRing) & 1, abort_v, p.status)) return;
+    const ItemDesc& d = descs[ds];
+    if (d.end) return;
+    // independent accumulator chains per 8-token tile so consecutive MMAs overlap
+    constexpr int NSET = NT8 >= 4 ? 1 : (4 / NT8);
+    float acc[NT8][NSET][4];
+#pragma unroll
+    for (int i = 0; i < NT8; ++i)
+#pragma unroll
+      for (int q = 0; q < NSET; ++q) acc[i][q][0] = acc[i][q][1] = acc[i][q][2] = acc[i][q][3] = 0.f;
+
+    for (int kt = grp; kt < KT; kt += 2) {
+      const uint32_t s = stage0 + kt;
+      const uint32_t slot = s % NSTAGE;
+      if (!mbar_wait(&full[slot], (s / NSTAGE) & 1, abort_v, p.status)) return;
+      // plain shared loads (ordered after the wait by its memory clobber) so the compiler
+      // can schedule them ahead of the dequantisation and the MMAs
+      const uint8_t* st = stages + slot * S::kStageBytes;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(st + S::kStageCodes + rb * 1024 + lane * 16);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(st + S::kStageCodes + rb * 1024 + 512 + lane * 16);
+      const uint4 sv = *reinterpret_cast<const uint4*>(st + S::kStageScales + rb * 128 + g * 16);
+      const uint8_t* act = st + S::kStageAct + g * kActPitch + t * 16;
+      const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+      const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};  // bf16 pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint16_t s0 = uint16_t(sw[j >> 1] >> (16 * (j & 1)));
+        const uint16_t s1 = uint16_t(sw[2 + (j >> 1)] >> (16 * (j & 1)));
+        uint32_t w0[4], w1[4];
+        dequant8(cw0[j], bf16_splat(s0), w0);
+        dequant8(cw1[j], bf16_splat(s1), w1);
+        const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
+        const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
+#pragma unroll
+        for (int n8 = 0; n8 < NT8; ++n8) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(act + n8 * 8 * kActPitch + j * 64);
+          mma_bf16_16816(acc[n8][j % NSET], a_lo, xv.x, xv.y);
+          mma_bf16_16816(acc[n8][(j + NSET / 2) % NSET], a_hi, xv.z, xv.w);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    float accs[NT8][4];
+#pragma unroll
+    for (int i = 0; i < NT8; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v = 0.f;
+#pragma unroll
+        for (int q = 0; q < NSET; ++q) v += acc[i][q][c];
+        accs[i][c] = v;
+      }
+    stage0 += KT;
+
+    // ---- hand over and epilogue
+    float* hw = handover + (rb * 32 + lane) * (4 * NT8);
+    if (grp == 1) {
+      if (it > 0 && !mbar_wait(hempty, (it - 1) & 1, abort_v, p.status)) return;
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8)
+        *reinterpret_cast<float4*>(hw + 4 * n8) = make_float4(accs[n8][0], accs[n8][1], accs[n8][2], accs[n8][3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(hfull);
+      continue;
+    }
+    if (!mbar_wait(hfull, it & 1, abort_v, p.status)) return;
+#pragma unroll
+    for (int n8 = 0; n8 < NT8; ++n8) {
+      const float4 o = *reinterpret_cast<const float4*>(hw + 4 * n8);
+      accs[n8][0] += o.x; accs[n8][1] += o.y; accs[n8][2] += o.z; accs[n8][3] += o.w;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(hempty);
+
+    if (EPI == kGateUp) {
+      const int i_col = d.nt * (kTileN / 2) + rb * 8 + g;  // intermediate column
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int col = n8 * 8 + 2 * t + q;
+          if (d.f[col] >= 0) {
+            const float v = silu_mul(accs[n8][q], accs[n8][2 + q]);
+            p.a_out[int64_t(d.pos0 + col) * p.I + i_col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          }
+        }
+      }
+    } else {
+      const int n0 = d.nt * kTileN + rb * 16 + g;
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int col = n8 * 8 + 2 * t + q;
+          const int f = d.f[col];
+          if (f >= 0) {
+            const float wgt = __ldg(p.topk_weights + f);
+            float* yr = p.y_out + int64_t(f) * p.H;
+            yr[n0] = accs[n8][q] * wgt;
+            yr[n0 + 8] = accs[n8][2 + q] * wgt;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&dempty[ds]);
+  }
+}
+
+template <int EPI, int TC>
+cudaError_t launch_one(const StreamParams& p, int grid, cudaStream_t stream) {
+  auto kern = stream_gemm_kernel<EPI, TC>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<TC>::kBytes);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kThreads, Smem<TC>::kBytes, stream>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_tc(const StreamParams& p, int tc, int grid, cudaStream_t stream) {
+  switch (tc) {
+    case 8: return launch_one<EPI, 8>(p, grid, stream);
+    case 16: return launch_one<EPI, 16>(p, grid, stream);
+    default: return launch_one<EPI, 32>(p, grid, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid) {
+  const int tc = a.block_m <= 8 ? 8 : (a.block_m <= 16 ? 16 : 32);
+  const int grid = a.num_sms;
+  StreamParams p{};
+  p.ntp = a.ntp;
+  p.sorted_ids = a.sorted_ids;
+  p.expert_ids = a.expert_ids;
+  p.block_m = a.block_m;
+  p.n_slots = a.T * a.topk;
+  p.topk = a.topk;
+  p.cap = a.cap;
+  p.a_out = a.a;
+  p.y_out = a.y;
+  p.topk_weights = a.topk_weights;
+  p.I = a.I;
+  p.H = a.H;
+  p.E = a.E;
+  p.status = a.status;
+
+  // gate_up: W13 [E, 2I, H], activations x [T, H]
+  p.blob = a.w13;
+  p.codes = reinterpret_cast<const uint32_t*>(a.w13 + blob_codes_offset());
+  p.scales = reinterpret_cast<const uint16_t*>(a.w13 + blob_scales_offset(a.E, 2 * a.I, a.H));
+  p.N = 2 * a.I;
+  p.K = a.H;
+  p.role = CHORD_ROLE_GATE_UP;
+  p.act = a.x;
+  p.act_ld = a.H;
+  cudaError_t err = launch_tc<kGateUp>(p, tc, grid, stream);
+  if (err != cudaSuccess) return err;
+  if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
+
+  // down: W2 [E, H, I], activations a [cap, I]
+  p.blob = a.w2;
+  p.codes = reinterpret_cast<const uint32_t*>(a.w2 + blob_codes_offset());
+  p.scales = reinterpret_cast<const uint16_t*>(a.w2 + blob_scales_offset(a.E, a.H, a.I));
+  p.N = a.H;
+  p.K = a.I;
+  p.role = CHORD_ROLE_DOWN;
+  p.act = a.a;
+  p.act_ld = a.I;
+  return launch_tc<kDown>(p, tc, grid, stream);
+}
+
+}  // namespace chord

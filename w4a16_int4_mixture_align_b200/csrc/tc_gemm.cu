@@ -1,0 +1,493 @@
+// tc_gemm.cu -- tensor-core (tcgen05) W4A16 grouped GEMMs for many tokens per expert.
+//
+// Above a few dozen routed tokens per expert the layer is bound by the tensor cores, and
+// the int4 dequantisation must be paid once per weight tile and shared by as many tokens
+// as possible. The Chord blog's H200 prefill kernels overlap the dequantisation of the
+// next K slice with the in-flight WGMMA group ("H200 Prefill und TP8": batched wait<1>
+// pipelining) and size block_m from the tokens routed per expert. On sm_100a the MMA is
+// asynchronous by construction, so the overlap becomes warp specialisation:
+//
+//   warp 0      producer: per item (routing block b of up to 256 rows, 128-row weight
+//               tile nt) one bulk copy of the packed codes + scales per 128-wide K step
+//               into a raw ring, and the routed activation rows of each 64-wide K step
+//               gathered by TMA (tile::gather4, 128-byte swizzle) into the B ring.
+//   warps 2..9  dequant: raw int4 -> bf16 (subtract 8, then scale) into the A ring in
+//               the UMMA K-major 128-byte-swizzle layout, 16 rows per warp.
+//   warp 1      MMA: one thread issues tcgen05.mma (M = 128 weight rows, N = the
+//               block's routed rows rounded up to 16, K = 16 per instruction) into one
+//               of two TMEM accumulators of 256 columns, and tcgen05.commit frees the
+//               ring stages and publishes the accumulator.
+//   warps 10..13 epilogue: tcgen05.ld of the accumulator; SiLU(gate)*up written to the
+//               bf16 intermediate (gate_up), or x topk_weight written to the per-slot
+//               fp32 buffer (down). Double buffering lets it overlap the next item.
+//
+// Operand orientation follows the blog's decode profile (dequantised weights in the
+// MMA-M slot, tokens in N): one dequantised weight tile serves every token of a block.
+// All waits are bounded; on timeout the CTA raises CHORD_DEV_TIMEOUT and unwinds after
+// waiting (bounded) for its copies and MMAs in flight, then frees TMEM.
+#include <cuda.h>
+
+#include "tc_common.cuh"
+
+namespace chord {
+namespace {
+
+constexpr int kRawStages = 4;
+constexpr int kABStages = 3;
+constexpr int kMaxN = 256;
+constexpr int kDescRingTC = 8;
+constexpr int kDequantWarps = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kTcThreads = 32 * (2 + kDequantWarps + kEpiWarps);
+
+constexpr int kAStageBytes = 128 * 64 * 2;
+constexpr int kBStageBytes = kMaxN * 64 * 2;
+constexpr int kRawStageBytes = kTileCodeBytes + kTileScaleBytes;
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kABStages * kAStageBytes;
+constexpr int kOffRaw = kOffB + kABStages * kBStageBytes;
+constexpr int kOffCoord = kOffRaw + kRawStages * kRawStageBytes;
+constexpr int kOffDesc = kOffCoord + kMaxN * 4;
+
+struct TcDesc {
+  int e, nt, pos0, nvalid, end, pad[3];
+};
+constexpr int kOffBar = kOffDesc + kDescRingTC * int(sizeof(TcDesc));
+constexpr int kNumBars = 2 * kRawStages + 3 * kABStages + 4 + 2 * kDescRingTC;
+constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kTcSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
+
+enum Epi { kGateUp = 0, kDown = 1 };
+
+struct TcParams {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const uint8_t* blob;
+  int N, K, E, role;
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntp;
+  int block_m;
+  int64_t n_slots;
+  int topk;
+  int64_t cap;
+  int act_rows;          // rows of the activation tensor map (out-of-range row = zero fill)
+  uint16_t* a_out;
+  float* y_out;
+  const float* topk_weights;
+  int I, H;
+  uint32_t* status;
+};
+
+// Dequantises half (64 K) of a raw 128x128 tile into an A stage: warp `rb` writes rows
+// rb*16 .. rb*16+15. Lane (g, t) converts the two words of K slices j = 2*hk, 2*hk+1 of
+// rows rb*16 + g and rb*16 + 8 + g; the slice order alternates with g so that the eight
+// lanes of each shared-memory phase hit eight distinct 16-byte bank groups.
+__device__ __forceinline__ void dequant_half(uint32_t raw, uint32_t a_stage, int rb, int hk, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint2 w = lds64(raw + rb * 1024 + h * 512 + g * 64 + t * 16 + hk * 8);
+    const uint32_t s = lds32(raw + kTileCodeBytes + rb * 128 + g * 16 + h * 8 + hk * 4);
+    const int r = rb * 16 + 8 * h + g;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int jj = (q + g) & 1;
+      uint32_t o[4];
+      dequant8(jj ? w.y : w.x, bf16_splat(uint16_t(jj ? (s >> 16) : (s & 0xFFFFu))), o);
+      const int c = 4 * jj + t;
+      sts128(a_stage + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4), o);
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled operand stages
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = raw_full + kRawStages;
+  uint64_t* a_full = raw_empty + kRawStages;
+  uint64_t* b_full = a_full + kABStages;
+  uint64_t* ab_empty = b_full + kABStages;
+  uint64_t* acc_full = ab_empty + kABStages;     // [2]
+  uint64_t* acc_empty = acc_full + 2;            // [2]
+  uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
+  uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
+  int* coords = reinterpret_cast<int*>(smem + kOffCoord);
+  TcDesc* descs = reinterpret_cast<TcDesc*>(smem + kOffDesc);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    const BlobHeader* hd = reinterpret_cast<const BlobHeader*>(p.blob);
+    if (hd->magic != kBlobMagic || hd->version != kBlobVersion || hd->layout != kLayoutTile128 ||
+        int(hd->role) != p.role || hd->E != p.E || hd->N != p.N || hd->K != p.K) {
+      abort_flag = 2;
+      if (blockIdx.x == 0) atomicOr(p.status, CHORD_DEV_BLOB_MISMATCH);
+    }
+    for (int s = 0; s < kRawStages; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], kDequantWarps);
+    }
+    for (int s = 0; s < kABStages; ++s) {
+      mbar_init(&a_full[s], kDequantWarps);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&ab_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    for (int d = 0; d < kDescRingTC; ++d) {
+      mbar_init(&dfull[d], 1);
+      mbar_init(&dempty[d], kDequantWarps + 1 + kEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (abort_flag) return;
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int* abort_v = &abort_flag;
+
+  const int KT = p.K / kTileK;        // 128-wide raw steps
+  const int NTILES = p.N / kTileN;
+
+  if (warp == 0) {
+    // ----------------------------------------------------------------- producer
+    int ntp = *p.ntp;
+    if (ntp < 0) ntp = 0;
+    if (ntp > p.cap) ntp = int(p.cap);
+    const int64_t nblocks = ntp / p.block_m;
+    const int64_t items = nblocks * NTILES;
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_a = policy_evict_last();
+    uint32_t rstage = 0, abstage = 0, nitem = 0;
+    bool ok = true;
+    for (int64_t w = blockIdx.x; ok; w += gridDim.x) {
+      const bool end = w >= items;
+      int e = -1, nt = 0, pos0 = 0, nvalid = 0;
+      if (!end) {
+        nt = int(w % NTILES);
+        const int64_t b = w / NTILES;
+        e = __ldg(p.expert_ids + b);
+        pos0 = int(b * p.block_m);
+        const bool e_ok = unsigned(e) < unsigned(p.E);
+        for (int r = lane; r < kMaxN; r += 32) {
+          int coord = p.act_rows;     // out of range: reads as zero
+          if (e_ok && r < p.block_m) {
+            const int f = __ldg(p.sorted_ids + pos0 + r);
+            if (f >= 0 && f < p.n_slots) {
+              coord = (EPI == kGateUp) ? f / p.topk : pos0 + r;
+              nvalid = r + 1;
+            }
+          }
+          coords[r] = coord;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
+        if (nvalid == 0) continue;
+      }
+      const uint32_t ds = nitem % kDescRingTC;
+      if (nitem >= kDescRingTC &&
+          !mbar_wait(&dempty[ds], ((nitem / kDescRingTC) - 1) & 1, abort_v, p.status))
+        break;
+      if (lane == 0) {
+        descs[ds].e = e;
+        descs[ds].nt = nt;
+        descs[ds].pos0 = pos0;
+        descs[ds].nvalid = nvalid;
+        descs[ds].end = end ? 1 : 0;
+        mbar_arrive(&dfull[ds]);
+      }
+      ++nitem;
+      if (end) break;
+      __syncwarp();
+      const int nmma = (nvalid + 15) & ~15;
+      const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const uint32_t rs = rstage % kRawStages;
+        if (rstage >= uint32_t(kRawStages) &&
+            !mbar_wait(&raw_empty[rs], ((rstage / kRawStages) - 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t* st = smem + kOffRaw + rs * kRawStageBytes;
+          mbar_arrive_expect_tx(&raw_full[rs], kRawStageBytes);
+          bulk_g2s_hint(st, p.codes + (tile0 + kt) * kTileCodeBytes, kTileCodeBytes, &raw_full[rs], pol_w);
+          bulk_g2s_hint(st + kTileCodeBytes, p.scales + (tile0 + kt) * kTileScaleBytes, kTileScaleBytes,
+                        &raw_full[rs], pol_w);
+        }
+        ++rstage;
+        for (int hk = 0; hk < 2; ++hk) {
+          const uint32_t s = abstage % kABStages;
+          if (abstage >= uint32_t(kABStages) &&
+              !mbar_wait(&ab_empty[s], ((abstage / kABStages) - 1) & 1, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
+          __syncwarp();
+          const uint32_t bst = sbase + kOffB + s * kBStageBytes;
+          const int col = kt * kTileK + hk * 64;
+          for (int i = lane; i < nmma / 4; i += 32)
+            tma_gather4(bst + i * 512, &tmap_act, col, coords[4 * i], coords[4 * i + 1],
+                        coords[4 * i + 2], coords[4 * i + 3], &b_full[s], pol_a);
+          ++abstage;
+        }
+      }
+      __syncwarp();
+    }
+    // drain: wait (bounded, ignoring abort) for the copies still in flight
+    if (lane == 0) {
+      int dummy = 0;
+      for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
+        mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
+      for (uint32_t s = (abstage > uint32_t(kABStages) ? abstage - kABStages : 0); s < abstage; ++s)
+        mbar_wait(&b_full[s % kABStages], (s / kABStages) & 1, &dummy, p.status);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t abstage = 0;
+      uint64_t* last_bar = nullptr;
+      uint32_t last_parity = 0;
+      for (uint32_t it = 0;; ++it) {
+        const uint32_t ds = it % kDescRingTC;
+        if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
+        const TcDesc d = descs[ds];
+        mbar_arrive(&dempty[ds]);
+        if (d.end) break;
+        const uint32_t buf = it & 1;
+        if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, abort_v, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * 256;
+        const uint32_t idesc = idesc_bf16_m128((d.nvalid + 15) & ~15);
+        bool ok = true;
+        for (int ks = 0; ks < 2 * KT; ++ks) {
+          const uint32_t s = abstage % kABStages, par = (abstage / kABStages) & 1;
+          if (!mbar_wait(&a_full[s], par, abort_v, p.status) || !mbar_wait(&b_full[s], par, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + kOffA + s * kAStageBytes;
+          const uint32_t b_addr = sbase + kOffB + s * kBStageBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
+                   (ks > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&ab_empty[s]);
+          last_bar = &ab_empty[s];
+          last_parity = par;
+          ++abstage;
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[buf]);
+      }
+      // make sure no MMA is still writing TMEM before it is freed
+      if (last_bar) {
+        int dummy = 0;
+        mbar_wait(last_bar, last_parity, &dummy, p.status);
+      }
+    }
+  } else if (warp < 2 + kDequantWarps) {
+    // ----------------------------------------------------------------- dequant
+    const int rb = warp - 2;
+    uint32_t rstage = 0, abstage = 0;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t ds = it % kDescRingTC;
+      if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
+      const int end = descs[ds].end;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[ds]);
+      if (end) break;
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const uint32_t rs = rstage % kRawStages;
+        if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
+        const uint32_t raw = sbase + kOffRaw + rs * kRawStageBytes;
+        for (int hk = 0; hk < 2; ++hk) {
+          const uint32_t s = abstage % kABStages;
+          if (abstage >= uint32_t(kABStages) &&
+              !mbar_wait(&ab_empty[s], ((abstage / kABStages) - 1) & 1, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          dequant_half(raw, sbase + kOffA + s * kAStageBytes, rb, hk, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
+          ++abstage;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
+        ++rstage;
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ----------------------------------------------------------------- epilogue
+    const int q = warp & 3;   // TMEM lane quadrant this warp may access
+    const int r = q * 32 + lane;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t ds = it % kDescRingTC;
+      if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
+      const TcDesc d = descs[ds];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[ds]);
+      if (d.end) break;
+      const uint32_t buf = it & 1;
+      if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_v, p.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * 256;
+      for (int c0 = 0; c0 < d.nvalid; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+        int f_l = -1;
+        float w_l = 0.f;
+        if (lane < 16 && c0 + lane < d.nvalid) {
+          const int f = __ldg(p.sorted_ids + d.pos0 + c0 + lane);
+          if (f >= 0 && f < p.n_slots) {
+            f_l = f;
+            if (EPI == kDown) w_l = __ldg(p.topk_weights + f);
+          }
+        }
+        if (EPI == kGateUp) {
+          const bool gate = (r & 15) < 8;
+          const int i_col = d.nt * (kTileN / 2) + (r >> 4) * 8 + (r & 7);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
+            const int f = __shfl_sync(0xffffffffu, f_l, c);
+            if (gate && f >= 0)
+              p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
+          }
+        } else {
+          const int n = d.nt * kTileN + r;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int f = __shfl_sync(0xffffffffu, f_l, c);
+            const float wgt = __shfl_sync(0xffffffffu, w_l, c);
+            if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c] * wgt;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------ host
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (row-major), box 64 columns x 1 row, 128-byte swizzle.
+cudaError_t make_row_gather_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int EPI>
+cudaError_t launch_one(const CUtensorMap& map, const TcParams& p, int grid, cudaStream_t stream) {
+  auto kern = tc_gemm_kernel<EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kTcThreads, kTcSmemBytes, stream>>>(map, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid) {
+  TcParams p{};
+  p.sorted_ids = a.sorted_ids;
+  p.expert_ids = a.expert_ids;
+  p.ntp = a.ntp;
+  p.block_m = a.block_m;
+  p.n_slots = a.T * a.topk;
+  p.topk = a.topk;
+  p.cap = a.cap;
+  p.a_out = a.a;
+  p.y_out = a.y;
+  p.topk_weights = a.topk_weights;
+  p.I = a.I;
+  p.H = a.H;
+  p.E = a.E;
+  p.status = a.status;
+  const int grid = a.num_sms;
+
+  // gate_up: W13 [E, 2I, H]; B rows gathered from x [T, H] by token
+  CUtensorMap map;
+  cudaError_t err = make_row_gather_map(&map, a.x, a.T, a.H);
+  if (err != cudaSuccess) return err;
+  p.blob = a.w13;
+  p.codes = a.w13 + blob_codes_offset();
+  p.scales = a.w13 + blob_scales_offset(a.E, 2 * a.I, a.H);
+  p.N = 2 * a.I;
+  p.K = a.H;
+  p.role = CHORD_ROLE_GATE_UP;
+  p.act_rows = int(a.T);
+  if ((err = launch_one<kGateUp>(map, p, grid, stream)) != cudaSuccess) return err;
+  if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
+
+  // down: W2 [E, H, I]; B rows of the intermediate a [cap, I] by sorted position
+  if ((err = make_row_gather_map(&map, a.a, a.cap, a.I)) != cudaSuccess) return err;
+  p.blob = a.w2;
+  p.codes = a.w2 + blob_codes_offset();
+  p.scales = a.w2 + blob_scales_offset(a.E, a.H, a.I);
+  p.N = a.H;
+  p.K = a.I;
+  p.role = CHORD_ROLE_DOWN;
+  p.act_rows = int(a.cap);
+  return launch_one<kDown>(map, p, grid, stream);
+}
+
+}  // namespace chord
