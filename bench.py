@@ -263,18 +263,15 @@ def run_chord(args, rank, world, local_rank):
     h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
     d2h = out_h.numel() * 2
 
-    # ---- max over ranks
-    stats = torch.tensor([elapsed_ms, e2e_ms, *seg_ms.tolist()], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(stats[0]), float(stats[1])
-    seg_ms = stats[2:].cpu().numpy()
+    # ---- max over ranks (outside the timed regions)
+    stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
+    elapsed_ms, e2e_ms = stats[0], stats[1]
+    seg_ms = np.array(stats[2:])
     if rank != 0:
         return None
 
     hbm, tf_burst, tf_sust, pk_kind = peaks()
-    us_call = elapsed_ms * 1000.0 / (K * world)
+    us_call = job_us_per_call(elapsed_ms, K, world)
     gu_us, dn_us = seg_ms[1] * 1000.0, seg_ms[2] * 1000.0
     decode = layer.block_m <= 32
     if decode:
@@ -309,12 +306,27 @@ def run_chord(args, rank, world, local_rank):
                   "hbm_frac": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9 / hbm, 4),
                   "TFLOP/s": round((work["gate_up_flops"] + work["down_flops"]) / (layer_us * 1e-6) / 1e12, 2)},
         "roofline": roofline,
-        "e2e": {"value": round(e2e_ms * 1000.0 / (K * world), 3), "unit": UNIT,
+        "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
     return line
+
+
+def max_over_ranks(vals, world, device=None):
+    """Element-wise max of `vals` over all ranks (one all-reduce; identity for world 1)."""
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def job_us_per_call(max_elapsed_ms: float, steps: int, world: int) -> float:
+    """Whole-job microseconds per layer call: every rank ran `steps` independent calls."""
+    return max_elapsed_ms * 1000.0 / (steps * world)
 
 
 def barrier(world):

@@ -6,13 +6,13 @@
 // those tensors deterministically: inside each expert the flat slot indices appear in
 // increasing order, so the result is a function of topk_ids alone.
 //
-// Work split: a warp owns a chunk of 1024 consecutive flat slots (32 per lane, loaded
-// up front so the loads overlap). Counting and ranking inside a chunk use
-// __match_any_sync over the expert ids of one 32-slot step: lanes with the same expert
-// get their rank from the popcount of lower peers, and the lowest peer advances the
-// expert's running position. Chunks are ordered by a prefix over chunk histograms.
+// Work split: a warp owns a run of consecutive 32-slot steps. Inside a step, the lanes
+// holding the same expert are found with one ballot per key bit; a lane's rank is the
+// popcount of its lower peers, and the lowest peer advances the expert's running
+// position. Runs are ordered by a prefix over per-run histograms.
 //
-//   n <= 32 chunks : one CTA of 32 warps does count, scan, scatter and fill (1 launch)
+//   n <= 32 x 1024 : one CTA of 32 warps (runs of ceil(n/1024) steps) does count, scan,
+//                    scatter and fill (1 launch)
 //   larger n       : count kernel (per-chunk histograms) -> scan kernel (1 CTA) ->
 //                    scatter + fill kernel, histograms in the caller's workspace.
 #include "chord_internal.cuh"
@@ -26,48 +26,71 @@ constexpr int kMaxE = 1024;
 
 __device__ __forceinline__ bool is_local(int e, int E) { return unsigned(e) < unsigned(E); }
 
-__device__ __forceinline__ void load_chunk(const int32_t* ids, int64_t n, int64_t c0, int v[kSteps]) {
+// Lanes of the warp holding the same key as this lane (key < 2^nbits), from one ballot
+// per key bit: cheaper than __match_any_sync when a step holds many distinct keys.
+__device__ __forceinline__ unsigned peers_of(unsigned key, int nbits) {
+  unsigned eq = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const unsigned bit = (key >> b) & 1u;
+    const unsigned m = __ballot_sync(0xffffffffu, bit);
+    eq &= bit ? m : ~m;
+  }
+  return eq;
+}
+
+__host__ __device__ inline int key_bits(int E) {
+  int b = 1;
+  while ((1 << b) <= E) ++b;  // keys 0..E fit in b bits
+  return b;
+}
+
+// Loads the ids of `steps` (<= kSteps) 32-slot steps starting at c0, all up front so the
+// loads overlap; slots past n read as -1 (not local).
+__device__ __forceinline__ void load_steps(const int32_t* ids, int64_t n, int64_t c0, int steps,
+                                           int v[kSteps]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
-    int64_t f = c0 + int64_t(s) * 32 + lane;
-    v[s] = f < n ? __ldg(ids + f) : -1;
+    const int64_t f = c0 + int64_t(s) * 32 + lane;
+    v[s] = (s < steps && f < n) ? __ldg(ids + f) : -1;
   }
 }
 
-// hist_row[e] += number of local slots of expert e in the chunk (warp-cooperative).
-__device__ __forceinline__ void chunk_count(const int v[kSteps], int E, int* hist_row) {
+// hist_row[e] += number of local slots of expert e among the loaded steps (warp-cooperative).
+// Non-local slots carry key E.
+__device__ __forceinline__ void chunk_count(const int v[kSteps], int steps, int E, int nbits,
+                                            int* hist_row) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
+    if (s >= steps) break;
     const int e = v[s];
     const bool loc = is_local(e, E);
-    const unsigned peers = __match_any_sync(0xffffffffu, loc ? unsigned(e) : 0xffffffffu);
+    const unsigned peers = peers_of(loc ? unsigned(e) : unsigned(E), nbits);
     if (loc && lane == __ffs(peers) - 1) hist_row[e] += __popc(peers);
     __syncwarp();
   }
 }
 
-// Places every local slot of the chunk at run_row[e] + (rank inside the expert),
+// Places every local slot of the loaded steps at run_row[e] + (rank inside the expert),
 // advancing run_row[e]. Ranks follow increasing flat index.
-__device__ __forceinline__ void chunk_scatter(const int v[kSteps], int64_t c0, int E, int* run_row,
-                                              int32_t* sorted_ids) {
+__device__ __forceinline__ void chunk_scatter(const int v[kSteps], int steps, int64_t c0, int E,
+                                              int nbits, int* run_row, int32_t* sorted_ids) {
   const int lane = threadIdx.x & 31;
   const unsigned lower = (1u << lane) - 1u;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
+    if (s >= steps) break;
     const int e = v[s];
     const bool loc = is_local(e, E);
-    const unsigned peers = __match_any_sync(0xffffffffu, loc ? unsigned(e) : 0xffffffffu);
-    if (loc) {
-      const int pos = run_row[e] + __popc(peers & lower);
-      sorted_ids[pos] = int32_t(c0 + int64_t(s) * 32 + lane);
-    }
+    const unsigned peers = peers_of(loc ? unsigned(e) : unsigned(E), nbits);
+    if (loc) sorted_ids[run_row[e] + __popc(peers & lower)] = int32_t(c0 + int64_t(s) * 32 + lane);
     __syncwarp();
     if (loc && lane == __ffs(peers) - 1) run_row[e] += __popc(peers);
     __syncwarp();
   }
 }
+
 
 // Exclusive prefix sum over vals[0..count) in shared memory (count <= blockDim.x <= 1024),
 // returns the total. All threads of the block must call it.
@@ -144,10 +167,13 @@ __global__ void __launch_bounds__(1024) align_single_kernel(
   for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
 
+  // warp w owns `steps` consecutive 32-slot steps, so every warp works even for small n
+  const int nbits = key_bits(E);
+  const int steps = int((n + 32 * 32 - 1) / (32 * 32));
+  const int64_t c0 = int64_t(warp) * steps * 32;
   int v[kSteps];
-  const int64_t c0 = int64_t(warp) * kChunk;
-  load_chunk(ids, n, c0, v);
-  if (c0 < n) chunk_count(v, E, hist + warp * E);
+  load_steps(ids, n, c0, steps, v);
+  if (c0 < n) chunk_count(v, steps, E, nbits, hist + warp * E);
   __syncthreads();
 
   for (int e = tid; e < E; e += blockDim.x) {
@@ -166,7 +192,7 @@ __global__ void __launch_bounds__(1024) align_single_kernel(
   for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] += off[i % E];
   __syncthreads();
 
-  if (c0 < n) chunk_scatter(v, c0, E, hist + warp * E, sorted_ids);
+  if (c0 < n) chunk_scatter(v, steps, c0, E, nbits, hist + warp * E, sorted_ids);
   fill_tail(cnt, off, E, block_m, n, cap, nblocks, sorted_ids, expert_ids, tid, blockDim.x);
   if (tid == 0) *ntp_out = off[E];
   if (offsets_out)
@@ -187,8 +213,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_count_kernel(
   const int64_t chunk = int64_t(blockIdx.x) * kWarpsPerCta + warp;
   if (chunk >= G) return;
   int v[kSteps];
-  load_chunk(ids, n, chunk * kChunk, v);
-  chunk_count(v, E, row);
+  load_steps(ids, n, chunk * kChunk, kSteps, v);
+  chunk_count(v, kSteps, E, key_bits(E), row);
   for (int e = lane; e < E; e += 32) chunk_hist[int64_t(e) * G + chunk] = row[e];
 }
 
@@ -237,8 +263,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
     for (int e = lane; e < E; e += 32) row[e] = off_g[e] + chunk_hist[int64_t(e) * G + chunk];
     __syncwarp();
     int v[kSteps];
-    load_chunk(ids, n, chunk * kChunk, v);
-    chunk_scatter(v, chunk * kChunk, E, row, sorted_ids);
+    load_steps(ids, n, chunk * kChunk, kSteps, v);
+    chunk_scatter(v, kSteps, chunk * kChunk, E, key_bits(E), row, sorted_ids);
   }
   fill_tail(cnt_g, off_g, E, block_m, n, cap, nblocks, sorted_ids, expert_ids,
             int64_t(blockIdx.x) * blockDim.x + threadIdx.x, int64_t(gridDim.x) * blockDim.x);

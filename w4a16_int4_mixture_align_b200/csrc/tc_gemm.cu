@@ -33,7 +33,8 @@ namespace chord {
 namespace {
 
 constexpr int kRawStages = 4;
-constexpr int kABStages = 3;
+constexpr int kAStages = 2;   // dequantised weights: produced on chip, double buffered
+constexpr int kBStages = 4;   // gathered activations: deep enough to cover TMA latency
 constexpr int kMaxN = 256;
 constexpr int kDescRingTC = 8;
 constexpr int kDequantWarps = 8;
@@ -44,8 +45,8 @@ constexpr int kAStageBytes = 128 * 64 * 2;
 constexpr int kBStageBytes = kMaxN * 64 * 2;
 constexpr int kRawStageBytes = kTileCodeBytes + kTileScaleBytes;
 constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kABStages * kAStageBytes;
-constexpr int kOffRaw = kOffB + kABStages * kBStageBytes;
+constexpr int kOffB = kOffA + kAStages * kAStageBytes;
+constexpr int kOffRaw = kOffB + kBStages * kBStageBytes;
 constexpr int kOffCoord = kOffRaw + kRawStages * kRawStageBytes;
 constexpr int kOffDesc = kOffCoord + kMaxN * 4;
 
@@ -53,7 +54,7 @@ struct TcDesc {
   int e, nt, pos0, nvalid, end, pad[3];
 };
 constexpr int kOffBar = kOffDesc + kDescRingTC * int(sizeof(TcDesc));
-constexpr int kNumBars = 2 * kRawStages + 3 * kABStages + 4 + 2 * kDescRingTC;
+constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 4 + 2 * kDescRingTC;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kTcSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
 
@@ -114,9 +115,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + kRawStages;
   uint64_t* a_full = raw_empty + kRawStages;
-  uint64_t* b_full = a_full + kABStages;
-  uint64_t* ab_empty = b_full + kABStages;
-  uint64_t* acc_full = ab_empty + kABStages;     // [2]
+  uint64_t* a_empty = a_full + kAStages;
+  uint64_t* b_full = a_empty + kAStages;
+  uint64_t* b_empty = b_full + kBStages;
+  uint64_t* acc_full = b_empty + kBStages;       // [2]
   uint64_t* acc_empty = acc_full + 2;            // [2]
   uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
   uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
@@ -138,10 +140,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kDequantWarps);
     }
-    for (int s = 0; s < kABStages; ++s) {
+    for (int s = 0; s < kAStages; ++s) {
       mbar_init(&a_full[s], kDequantWarps);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&ab_empty[s], 1);
+      mbar_init(&b_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t items = nblocks * NTILES;
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
-    uint32_t rstage = 0, abstage = 0, nitem = 0;
+    uint32_t rstage = 0, bstage = 0, nitem = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok; w += gridDim.x) {
       const bool end = w >= items;
@@ -233,9 +238,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ++rstage;
         for (int hk = 0; hk < 2; ++hk) {
-          const uint32_t s = abstage % kABStages;
-          if (abstage >= uint32_t(kABStages) &&
-              !mbar_wait(&ab_empty[s], ((abstage / kABStages) - 1) & 1, abort_v, p.status)) {
+          const uint32_t s = bstage % kBStages;
+          if (bstage >= uint32_t(kBStages) &&
+              !mbar_wait(&b_empty[s], ((bstage / kBStages) - 1) & 1, abort_v, p.status)) {
             ok = false;
             break;
           }
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = lane; i < nmma / 4; i += 32)
             tma_gather4(bst + i * 512, &tmap_act, col, coords[4 * i], coords[4 * i + 1],
                         coords[4 * i + 2], coords[4 * i + 3], &b_full[s], pol_a);
-          ++abstage;
+          ++bstage;
         }
       }
       __syncwarp();
@@ -256,8 +261,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int dummy = 0;
       for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
         mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
-      for (uint32_t s = (abstage > uint32_t(kABStages) ? abstage - kABStages : 0); s < abstage; ++s)
-        mbar_wait(&b_full[s % kABStages], (s / kABStages) & 1, &dummy, p.status);
+      for (uint32_t s = (bstage > uint32_t(kBStages) ? bstage - kBStages : 0); s < bstage; ++s)
+        mbar_wait(&b_full[s % kBStages], (s / kBStages) & 1, &dummy, p.status);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
@@ -278,21 +283,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t idesc = idesc_bf16_m128((d.nvalid + 15) & ~15);
         bool ok = true;
         for (int ks = 0; ks < 2 * KT; ++ks) {
-          const uint32_t s = abstage % kABStages, par = (abstage / kABStages) & 1;
-          if (!mbar_wait(&a_full[s], par, abort_v, p.status) || !mbar_wait(&b_full[s], par, abort_v, p.status)) {
+          const uint32_t sa = abstage % kAStages, pa = (abstage / kAStages) & 1;
+          const uint32_t sb = abstage % kBStages, pb = (abstage / kBStages) & 1;
+          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status) || !mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = sbase + kOffA + s * kAStageBytes;
-          const uint32_t b_addr = sbase + kOffB + s * kBStageBytes;
+          const uint32_t a_addr = sbase + kOffA + sa * kAStageBytes;
+          const uint32_t b_addr = sbase + kOffB + sb * kBStageBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
                    (ks > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&ab_empty[s]);
-          last_bar = &ab_empty[s];
-          last_parity = par;
+          tc_commit(&a_empty[sa]);
+          tc_commit(&b_empty[sb]);
+          last_bar = &b_empty[sb];
+          last_parity = pb;
           ++abstage;
         }
         if (!ok) break;
@@ -321,9 +328,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
         const uint32_t raw = sbase + kOffRaw + rs * kRawStageBytes;
         for (int hk = 0; hk < 2; ++hk) {
-          const uint32_t s = abstage % kABStages;
-          if (abstage >= uint32_t(kABStages) &&
-              !mbar_wait(&ab_empty[s], ((abstage / kABStages) - 1) & 1, abort_v, p.status)) {
+          const uint32_t s = abstage % kAStages;
+          if (abstage >= uint32_t(kAStages) &&
+              !mbar_wait(&a_empty[s], ((abstage / kAStages) - 1) & 1, abort_v, p.status)) {
             ok = false;
             break;
           }
