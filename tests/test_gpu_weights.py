@@ -33,22 +33,22 @@ def repack(chord, qw, s, role):
 
 
 def invert_layout(blob: np.ndarray, E, N, K, role):
-    """Numpy inverse of the tile layout -> (qweight [E,N,K/8] int32, scales [E,N,K/32] u16)."""
-    codes_off = 256
-    scales_off = (256 + E * N * K // 2 + 255) // 256 * 256
+    """Numpy inverse of the tile layout -> (qweight [E,N,K/8] int32, scales [E,N,K/32] u16).
+
+    Tiles of 9216 bytes after a 256-byte header, tile (e, nt, kt) in that order; each
+    tile is 8192 bytes of codes then 1024 bytes of scales."""
     NT, KT = N // 128, K // 128
-    codes = blob[codes_off:codes_off + E * N * K // 2].view(np.uint32)
+    tiles = blob[256:256 + E * NT * KT * 9216].reshape(E, NT, KT, 9216)
+    codes = np.ascontiguousarray(tiles[..., :8192]).view(np.uint32)
     codes = codes.reshape(E, NT, KT, 8, 2, 8, 4, 4)          # e nt kt rb h g t j
     # un-permute nibbles: K offset u sits in nibble (u>>1) + 4*(u&1)
     slot = [(u >> 1) + 4 * (u & 1) for u in range(8)]
-    nib = np.stack([(codes >> np.uint32(4 * slot[u])) & np.uint32(0xF) for u in range(8)], axis=-1)
     words = np.zeros(codes.shape, dtype=np.uint32)
     for u in range(8):
-        words |= nib[..., u] << np.uint32(4 * u)
+        words |= ((codes >> np.uint32(4 * slot[u])) & np.uint32(0xF)) << np.uint32(4 * u)
     # physical row p = nt*128 + rb*16 + 8h + g ; k/8 = kt*16 + 4j + t
-    w = words.transpose(0, 1, 3, 4, 5, 2, 7, 6)               # e nt rb h g kt j t
-    w = w.reshape(E, N, K // 8)
-    sc = blob[scales_off:scales_off + E * N * K // 32 * 2].view(np.uint16)
+    w = words.transpose(0, 1, 3, 4, 5, 2, 7, 6).reshape(E, N, K // 8)
+    sc = np.ascontiguousarray(tiles[..., 8192:]).view(np.uint16)
     sc = sc.reshape(E, NT, KT, 8, 8, 2, 4)                     # e nt kt rb g h j
     sc = sc.transpose(0, 1, 3, 5, 4, 2, 6).reshape(E, N, K // 32)
     if role == 1:  # gate_up: physical block of 16 = 8 gate rows then 8 up rows
@@ -70,7 +70,7 @@ def test_repack_layout_round_trip(chord, role, E, N, K):
     s = rng.integers(0, 2 ** 16, size=(E, N, K // 32), dtype=np.uint16)
     blob = repack(chord, qw, s, role).cpu().numpy()
     hdr = blob[:48].view(np.uint32)
-    assert hdr[0] == 0x34574843 and hdr[1] == 1 and hdr[3] == role
+    assert hdr[0] == 0x34574843 and hdr[1] == 2 and hdr[2] == 2 and hdr[3] == role
     assert list(hdr[4:8].view(np.int32)) == [E, N, K, 32]
     qw2, s2 = invert_layout(blob, E, N, K, role)
     assert np.array_equal(qw2, qw)

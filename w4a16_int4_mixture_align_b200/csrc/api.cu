@@ -281,6 +281,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   a.out = out;
   a.a = reinterpret_cast<uint16_t*>(wsb + ws.a_offset);
   a.y = reinterpret_cast<float*>(wsb + ws.y_offset);
+  a.xs = reinterpret_cast<uint16_t*>(wsb + ws.xs_offset);
   a.status = reinterpret_cast<uint32_t*>(wsb);
   a.T = T;
   a.H = H;

@@ -3,12 +3,15 @@
 // Repacked weight blob (written by chord_repack_weights, read by the GEMM kernels):
 //
 //   [0, 256)        BlobHeader
-//   codes           E * N * K / 2 bytes, 256-byte aligned
-//   scales          E * N * (K/32) * 2 bytes, 256-byte aligned
+//   tiles           E * (N/128) * (K/128) tiles of 9216 bytes, tile (e, nt, kt) at
+//                   256 + ((e * N/128 + nt) * K/128 + kt) * 9216
 //
-// Codes are grouped in tiles of 128 physical rows x 128 K (8 KiB), tile (e, nt, kt)
-// at byte ((e * N/128 + nt) * K/128 + kt) * 8192. A tile is 8 sub-tiles of 16 rows
-// (rb = 0..7, 1 KiB each). Inside a sub-tile the int32 word index is
+// A tile covers 128 physical rows x 128 K: 8192 bytes of int4 codes followed by the
+// 1024 bytes of their bf16 scales, so consecutive K tiles of one row block form one
+// contiguous run that a single bulk copy brings in.
+//
+// Codes: 8 sub-tiles of 16 rows (rb = 0..7, 1 KiB each). Inside a sub-tile the int32
+// word index is
 //     h*128 + g*16 + t*4 + j         (h 0..1, g 0..7, t 0..3, j 0..3)
 // and holds physical row  rb*16 + 8h + g  and K range  kt*128 + 32j + 8t + [0, 8).
 // Lane (g, t) of a warp therefore reads its two 16-byte vectors (h = 0, 1) from
@@ -16,8 +19,8 @@
 // (u >> 1) + 4 * (u & 1), so that masking nibbles {i, i+4} after a right shift by 4i
 // yields the bf16 pair (u = 2i, 2i+1) in order.
 //
-// Scales are tiled the same way: 1 KiB per tile, 128 bytes per sub-tile, bf16 index
-//     g*8 + h*4 + j      for physical row rb*16 + 8h + g, group kt*4 + j.
+// Scales: 128 bytes per sub-tile, bf16 index  g*8 + h*4 + j  for physical row
+// rb*16 + 8h + g, group kt*4 + j.
 //
 // Physical row p maps to a logical row: for the down projection p itself; for gate_up
 // (N = 2I) block p/16 holds gate rows 8*(p/16) + [0, 8) followed by the matching up
@@ -34,13 +37,14 @@
 namespace chord {
 
 constexpr uint32_t kBlobMagic = 0x34574843u;  // "CHW4"
-constexpr uint32_t kBlobVersion = 1;
-constexpr uint32_t kLayoutTile128 = 1;
+constexpr uint32_t kBlobVersion = 2;
+constexpr uint32_t kLayoutTile128 = 2;  // 128x128 tiles, scales interleaved after codes
 constexpr int kGroup = 32;
 constexpr int kTileN = 128;
 constexpr int kTileK = 128;
 constexpr int kTileCodeBytes = kTileN * kTileK / 2;          // 8192
 constexpr int kTileScaleBytes = kTileN * (kTileK / kGroup) * 2;  // 1024
+constexpr int kTileBytes = kTileCodeBytes + kTileScaleBytes;     // 9216
 constexpr int kHeaderBytes = 256;
 
 struct BlobHeader {
@@ -49,8 +53,8 @@ struct BlobHeader {
   uint32_t layout;
   uint32_t role;
   int32_t E, N, K, group;
-  uint64_t codes_offset;
-  uint64_t scales_offset;
+  uint64_t tiles_offset;
+  uint64_t tile_bytes;
   uint64_t total_bytes;
   uint32_t reserved[50];
 };
@@ -58,18 +62,12 @@ static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
 
 __host__ __device__ inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
-__host__ __device__ inline uint64_t blob_codes_bytes(int E, int N, int K) {
-  return uint64_t(E) * N * (K / 2);
-}
-__host__ __device__ inline uint64_t blob_scales_bytes(int E, int N, int K) {
-  return uint64_t(E) * N * (K / kGroup) * 2;
-}
-__host__ __device__ inline uint64_t blob_codes_offset() { return kHeaderBytes; }
-__host__ __device__ inline uint64_t blob_scales_offset(int E, int N, int K) {
-  return align256(kHeaderBytes + blob_codes_bytes(E, N, K));
+__host__ __device__ inline uint64_t blob_tiles_offset() { return kHeaderBytes; }
+__host__ __device__ inline uint64_t blob_num_tiles(int E, int N, int K) {
+  return uint64_t(E) * (N / kTileN) * (K / kTileK);
 }
 __host__ __device__ inline uint64_t blob_total_bytes(int E, int N, int K) {
-  return align256(blob_scales_offset(E, N, K) + blob_scales_bytes(E, N, K));
+  return align256(kHeaderBytes + blob_num_tiles(E, N, K) * kTileBytes);
 }
 
 // Logical row of physical row p in a tile-layout matrix with N physical rows.
@@ -83,9 +81,12 @@ __host__ __device__ inline int logical_row(int role, int N, int p) {
 __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1); }
 
 // ------------------------------------------------------------------------------------
-// Workspace of chord_moe_forward: [status 256 B][a: cap x I bf16][y: T*topk x H fp32]
+// Workspace of chord_moe_forward:
+//   [status 256 B][a: cap x I bf16][y: T*topk x H fp32][xs: cap x H bf16]
+// a is the SiLU*up intermediate by sorted position, y the weighted expert outputs by
+// flat slot, xs the hidden rows in sorted order (tensor-core schedule only).
 struct ForwardWorkspace {
-  uint64_t a_offset, y_offset, total;
+  uint64_t a_offset, y_offset, xs_offset, total;
 };
 __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int topk, int E, int H,
                                                               int I, int block_m) {
@@ -93,7 +94,8 @@ __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int top
   int64_t cap = T * topk + int64_t(E) * (block_m - 1);
   w.a_offset = 256;
   w.y_offset = align256(w.a_offset + uint64_t(cap) * I * 2);
-  w.total = align256(w.y_offset + uint64_t(T) * topk * H * 4);
+  w.xs_offset = align256(w.y_offset + uint64_t(T) * topk * H * 4);
+  w.total = align256(w.xs_offset + uint64_t(cap) * H * 2);
   return w;
 }
 
@@ -280,6 +282,7 @@ struct ForwardArgs {
   uint16_t* out;
   uint16_t* a;     // [cap, I] bf16 intermediate, indexed by sorted position
   float* y;        // [T*topk, H] fp32 weighted expert outputs, indexed by flat slot
+  uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
   uint32_t* status;
   int64_t T;
   int H, I, E, topk, block_m;

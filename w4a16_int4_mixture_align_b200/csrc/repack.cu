@@ -18,9 +18,9 @@ __device__ __forceinline__ uint32_t permute_nibbles(uint32_t src) {
   return out;
 }
 
-// One thread per repacked code word.
+// One thread per repacked code word; `tiles` is the blob's tile region.
 __global__ void repack_codes_kernel(const int32_t* __restrict__ qweight, int E, int N, int K,
-                                    int role, uint32_t* __restrict__ codes) {
+                                    int role, uint8_t* __restrict__ tiles) {
   const int NT = N / kTileN, KT = K / kTileK;
   const int64_t total = int64_t(E) * N * (K / 8);
   for (int64_t w = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
@@ -36,13 +36,13 @@ __global__ void repack_codes_kernel(const int32_t* __restrict__ qweight, int E, 
     const int n = logical_row(role, N, p);
     const int k0 = kt * kTileK + 32 * j + 8 * t;
     const uint32_t src = uint32_t(qweight[(int64_t(e) * N + n) * (K / 8) + k0 / 8]);
-    codes[w] = permute_nibbles(src);
+    reinterpret_cast<uint32_t*>(tiles + tile * kTileBytes)[w & 2047] = permute_nibbles(src);
   }
 }
 
 // One thread per repacked scale.
 __global__ void repack_scales_kernel(const uint16_t* __restrict__ scales, int E, int N, int K,
-                                     int role, uint16_t* __restrict__ out) {
+                                     int role, uint8_t* __restrict__ tiles) {
   const int NT = N / kTileN, KT = K / kTileK;
   const int64_t total = int64_t(E) * N * (K / kGroup);
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -55,7 +55,8 @@ __global__ void repack_scales_kernel(const uint16_t* __restrict__ scales, int E,
     const int e = int(rest / NT);
     const int p = nt * kTileN + rb * 16 + 8 * h + g;
     const int n = logical_row(role, N, p);
-    out[i] = scales[(int64_t(e) * N + n) * (K / kGroup) + kt * 4 + j];
+    reinterpret_cast<uint16_t*>(tiles + tile * kTileBytes + kTileCodeBytes)[i & 511] =
+        scales[(int64_t(e) * N + n) * (K / kGroup) + kt * 4 + j];
   }
 }
 
@@ -72,8 +73,8 @@ __global__ void write_header_kernel(uint8_t* blob, int E, int N, int K, int role
     hd->N = N;
     hd->K = K;
     hd->group = kGroup;
-    hd->codes_offset = blob_codes_offset();
-    hd->scales_offset = blob_scales_offset(E, N, K);
+    hd->tiles_offset = blob_tiles_offset();
+    hd->tile_bytes = kTileBytes;
     hd->total_bytes = blob_total_bytes(E, N, K);
   }
 }
@@ -83,8 +84,7 @@ __global__ void write_header_kernel(uint8_t* blob, int E, int N, int K, int role
 __global__ void dequant_blob_kernel(const uint8_t* __restrict__ blob, int E, int N, int K, int role,
                                     uint16_t* __restrict__ w) {
   const int NT = N / kTileN, KT = K / kTileK;
-  const uint32_t* codes = reinterpret_cast<const uint32_t*>(blob + blob_codes_offset());
-  const uint16_t* scales = reinterpret_cast<const uint16_t*>(blob + blob_scales_offset(E, N, K));
+  const uint8_t* tiles = blob + blob_tiles_offset();
   const int64_t total = int64_t(E) * N * (K / 8);
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
@@ -98,9 +98,10 @@ __global__ void dequant_blob_kernel(const uint8_t* __restrict__ blob, int E, int
     const int p = nt * kTileN + rb * 16 + 8 * h + g;
     const int n = logical_row(role, N, p);
     const int k0 = kt * kTileK + 32 * j + 8 * t;
-    const uint16_t s = scales[tile * (kTileScaleBytes / 2) + rb * 64 + g * 8 + h * 4 + j];
+    const uint8_t* tp = tiles + tile * kTileBytes;
+    const uint16_t s = reinterpret_cast<const uint16_t*>(tp + kTileCodeBytes)[rb * 64 + g * 8 + h * 4 + j];
     uint32_t pairs[4];
-    dequant8(codes[i], bf16_splat(s), pairs);
+    dequant8(reinterpret_cast<const uint32_t*>(tp)[i & 2047], bf16_splat(s), pairs);
     uint4 v = make_uint4(pairs[0], pairs[1], pairs[2], pairs[3]);
     *reinterpret_cast<uint4*>(w + (int64_t(e) * N + n) * K + k0) = v;
   }
@@ -118,11 +119,11 @@ cudaError_t launch_repack(const int32_t* qweight, const uint16_t* scales, int E,
                           int role, uint8_t* blob, cudaStream_t stream) {
   write_header_kernel<<<1, 64, 0, stream>>>(blob, E, N, K, role);
   const int64_t words = int64_t(E) * N * (K / 8);
-  repack_codes_kernel<<<grid_for(words, 256), 256, 0, stream>>>(
-      qweight, E, N, K, role, reinterpret_cast<uint32_t*>(blob + blob_codes_offset()));
+  repack_codes_kernel<<<grid_for(words, 256), 256, 0, stream>>>(qweight, E, N, K, role,
+                                                                 blob + blob_tiles_offset());
   const int64_t nsc = int64_t(E) * N * (K / kGroup);
-  repack_scales_kernel<<<grid_for(nsc, 256), 256, 0, stream>>>(
-      scales, E, N, K, role, reinterpret_cast<uint16_t*>(blob + blob_scales_offset(E, N, K)));
+  repack_scales_kernel<<<grid_for(nsc, 256), 256, 0, stream>>>(scales, E, N, K, role,
+                                                                blob + blob_tiles_offset());
   count_launches(3);
   return cudaGetLastError();
 }

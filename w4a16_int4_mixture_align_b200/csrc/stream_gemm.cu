@@ -7,13 +7,15 @@
 // weight tiles streamed by bulk asynchronous copies through a deep shared-memory ring:
 //
 //   warp 0        producer: per item (routing block b, token chunk c, 128-row tile nt)
-//                 it publishes a descriptor, then per 128-wide K step issues one 8 KiB
-//                 code copy, one 1 KiB scale copy and one 256-byte copy per routed
-//                 activation row, all completing on the stage's mbarrier.
-//   warps 1..8    consumer group 0, warps 9..16 group 1: group g takes the K steps of
-//                 parity g; warp w owns 16 physical rows. Codes go shared -> registers,
-//                 dequantise to bf16 pairs (subtract 8, then scale) that are exactly the
-//                 A fragments of mma.m16n8k16; tokens are the N dimension.
+//                 it publishes a descriptor, then per stage of KTS consecutive 128-wide
+//                 K tiles issues ONE bulk copy of their codes + scales (up to 36 KiB:
+//                 a bulk copy has a high fixed cost, so bytes per copy decide the
+//                 streaming rate) and cp.async copies of the routed activation rows,
+//                 all completing on the stage's mbarrier.
+//   warps 1..8    consumer group 0, warps 9..16 group 1: group g takes the tiles of
+//                 parity g inside each stage; warp w owns 16 physical rows. Codes go
+//                 shared -> registers and dequantise to bf16 pairs (subtract 8, then
+//                 scale) that are exactly the A fragments of mma.m16n8k16; tokens are N.
 //   epilogue      group 1 hands its partial sums to group 0, which adds them and applies
 //                 SiLU(gate)*up (gate_up; gate and up rows are interleaved by the repack)
 //                 or the top-k weight (down, written to the per-slot buffer y).
@@ -27,15 +29,13 @@ namespace {
 
 constexpr int kConsumerWarps = 16;          // two groups of 8
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
-constexpr int kActPitch = 320;              // bytes per activation row in a stage (256 + 64 pad)
 constexpr int kDescRing = 32;
 constexpr int kMaxTC = 32;
 
 enum Epi { kGateUp = 0, kDown = 1 };
 
 struct StreamParams {
-  const uint32_t* codes;    // blob codes region
-  const uint16_t* scales;   // blob scales region
+  const uint8_t* tiles;     // blob tile region
   const uint8_t* blob;      // header
   int N, K;                 // physical rows, reduction length
   int E, role;
@@ -62,25 +62,34 @@ struct ItemDesc {
 
 template <int TC>
 struct Smem {
-  static constexpr int kStageCodes = 0;
-  static constexpr int kStageScales = kTileCodeBytes;
-  static constexpr int kStageAct = kTileCodeBytes + kTileScaleBytes;
+  static constexpr int kKTS = TC <= 16 ? 4 : 2;                 // K tiles per stage
+  static constexpr int kStageAct = kKTS * kTileBytes;           // activation rows after the tiles
+  static constexpr int kActPitch = kKTS * 256 + 64;             // padded row pitch (bank spread)
   static constexpr int kStageBytes = ((kStageAct + TC * kActPitch) + 127) / 128 * 128;
   static constexpr int kHandoverBytes = 8 * 32 * (TC / 8) * 4 * 4;  // 8 warps x 32 lanes x 4*NT floats
   static constexpr int kBudget = 200 * 1024;
   static constexpr int kFit =
       (kBudget - kHandoverBytes - kDescRing * int(sizeof(ItemDesc)) - 1024) / kStageBytes;
-  static constexpr int kStages = kFit > 24 ? 24 : kFit;
+  static constexpr int kStages = kFit > 12 ? 12 : kFit;
   static constexpr int kBytes =
       kStages * kStageBytes + kHandoverBytes + kDescRing * int(sizeof(ItemDesc)) + 1024;
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrives on `bar` once this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 template <int EPI, int TC>
 __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p) {
   using S = Smem<TC>;
   constexpr int NT8 = TC / 8;
   constexpr int NSTAGE = S::kStages;
-  static_assert(NSTAGE >= 4 && NSTAGE < kDescRing, "stage count");
+  constexpr int KTS = S::kKTS;
+  static_assert(NSTAGE >= 3 && NSTAGE < kDescRing, "stage count");
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stages = smem;
   float* handover = reinterpret_cast<float*>(smem + NSTAGE * S::kStageBytes);
@@ -105,8 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       if (blockIdx.x == 0) atomicOr(p.status, CHORD_DEV_BLOB_MISMATCH);
     }
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 8);
+      mbar_init(&full[s], 1 + 32);  // producer expect_tx + one cp.async arrival per lane
+      mbar_init(&empty[s], kConsumerWarps);
     }
     for (int s = 0; s < kDescRing; ++s) {
       mbar_init(&dfull[s], 1);
@@ -121,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
   volatile int* abort_v = &abort_flag;
 
   const int KT = p.K / kTileK;
+  const int KS = (KT + KTS - 1) / KTS;         // stages per item
   const int NTILES = p.N / kTileN;
   const int cpb = (p.block_m + TC - 1) / TC;  // token chunks per routing block
 
@@ -167,38 +177,43 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       if (lane == 0) mbar_arrive(&dfull[ds]);
       ++nitem;
       if (end) break;
-      // stream the item's K steps
-      const unsigned rows = __ballot_sync(0xffffffffu, fval >= 0);
-      const uint32_t bytes = kTileCodeBytes + kTileScaleBytes + __popc(rows) * 256u;
+      // stream the item: one bulk copy of KTS tiles (codes + scales) per stage, and the
+      // routed activation rows by cp.async (16 B per lane per copy)
       const int64_t act_row = (EPI == kGateUp) ? int64_t(fval / p.topk) : int64_t(pos0 + lane);
       const uint16_t* act_src = p.act + act_row * p.act_ld;
       const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
       bool ok = true;
-      for (int kt = 0; kt < KT; ++kt, ++stage) {
+      for (int ks = 0; ks < KS; ++ks, ++stage) {
         const uint32_t slot = stage % NSTAGE;
         if (stage >= uint32_t(NSTAGE) &&
             !mbar_wait(&empty[slot], ((stage / NSTAGE) - 1) & 1, abort_v, p.status)) {
           ok = false;
           break;
         }
+        const int kt0 = ks * KTS;
+        const int ntl = min(KTS, KT - kt0);
         uint8_t* st = stages + slot * S::kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
-        __syncwarp();
         if (lane == 0) {
-          bulk_g2s_hint(st + S::kStageCodes,
-                        reinterpret_cast<const uint8_t*>(p.codes) + (tile0 + kt) * kTileCodeBytes,
-                        kTileCodeBytes, &full[slot], pol_w);
-          bulk_g2s_hint(st + S::kStageScales,
-                        reinterpret_cast<const uint8_t*>(p.scales) + (tile0 + kt) * kTileScaleBytes,
-                        kTileScaleBytes, &full[slot], pol_w);
+          mbar_arrive_expect_tx(&full[slot], uint32_t(ntl) * kTileBytes);
+          bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &full[slot],
+                        pol_w);
         }
-        if (fval >= 0)
-          bulk_g2s_hint(st + S::kStageAct + lane * kActPitch, act_src + kt * kTileK, 256,
-                        &full[slot], pol_a);
+        const int chunks_per_row = ntl * 16;
+        const uint32_t act_base = smem_u32(st + S::kStageAct);
+        for (int c = lane; c < TC * 16 * KTS; c += 32) {
+          const int r = c / (16 * KTS), q = c % (16 * KTS);
+          const int f = __shfl_sync(0xffffffffu, fval, r);
+          const uint16_t* src = reinterpret_cast<const uint16_t*>(
+              __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(act_src), r));
+          if (f >= 0 && q < chunks_per_row)
+            cp_async16(act_base + r * S::kActPitch + q * 16, src + kt0 * kTileK + q * 8);
+        }
+        cp_async_arrive(&full[slot]);
       }
       if (!ok) break;
     }
     // drain: wait (bounded, ignoring the abort flag) for every copy still in flight
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       int dummy = 0;
       const uint32_t first = stage > uint32_t(NSTAGE) ? stage - NSTAGE : 0;
@@ -227,34 +242,38 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 #pragma unroll
       for (int q = 0; q < NSET; ++q) acc[i][q][0] = acc[i][q][1] = acc[i][q][2] = acc[i][q][3] = 0.f;
 
-    for (int kt = grp; kt < KT; kt += 2) {
-      const uint32_t s = stage0 + kt;
+    for (int ks = 0; ks < KS; ++ks) {
+      const uint32_t s = stage0 + ks;
       const uint32_t slot = s % NSTAGE;
       if (!mbar_wait(&full[slot], (s / NSTAGE) & 1, abort_v, p.status)) return;
+      const int ntl = min(KTS, KT - ks * KTS);
       // plain shared loads (ordered after the wait by its memory clobber) so the compiler
       // can schedule them ahead of the dequantisation and the MMAs
-      const uint8_t* st = stages + slot * S::kStageBytes;
-      const uint4 c0 = *reinterpret_cast<const uint4*>(st + S::kStageCodes + rb * 1024 + lane * 16);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(st + S::kStageCodes + rb * 1024 + 512 + lane * 16);
-      const uint4 sv = *reinterpret_cast<const uint4*>(st + S::kStageScales + rb * 128 + g * 16);
-      const uint8_t* act = st + S::kStageAct + g * kActPitch + t * 16;
-      const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
-      const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};  // bf16 pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
+      const uint8_t* stg = stages + slot * S::kStageBytes;
+      for (int i = grp; i < ntl; i += 2) {
+        const uint8_t* st = stg + i * kTileBytes;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
+        const uint4 sv = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + g * 16);
+        const uint8_t* act = stg + S::kStageAct + g * S::kActPitch + i * 256 + t * 16;
+        const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+        const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};  // bf16 pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint16_t s0 = uint16_t(sw[j >> 1] >> (16 * (j & 1)));
-        const uint16_t s1 = uint16_t(sw[2 + (j >> 1)] >> (16 * (j & 1)));
-        uint32_t w0[4], w1[4];
-        dequant8(cw0[j], bf16_splat(s0), w0);
-        dequant8(cw1[j], bf16_splat(s1), w1);
-        const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
-        const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
+        for (int j = 0; j < 4; ++j) {
+          const uint16_t s0 = uint16_t(sw[j >> 1] >> (16 * (j & 1)));
+          const uint16_t s1 = uint16_t(sw[2 + (j >> 1)] >> (16 * (j & 1)));
+          uint32_t w0[4], w1[4];
+          dequant8(cw0[j], bf16_splat(s0), w0);
+          dequant8(cw1[j], bf16_splat(s1), w1);
+          const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
+          const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
 #pragma unroll
-        for (int n8 = 0; n8 < NT8; ++n8) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(act + n8 * 8 * kActPitch + j * 64);
-          mma_bf16_16816(acc[n8][j % NSET], a_lo, xv.x, xv.y);
-          mma_bf16_16816(acc[n8][(j + NSET / 2) % NSET], a_hi, xv.z, xv.w);
+          for (int n8 = 0; n8 < NT8; ++n8) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(act + n8 * 8 * S::kActPitch + j * 64);
+            mma_bf16_16816(acc[n8][j % NSET], a_lo, xv.x, xv.y);
+            mma_bf16_16816(acc[n8][(j + NSET / 2) % NSET], a_hi, xv.z, xv.w);
+          }
         }
       }
       __syncwarp();
@@ -270,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
         for (int q = 0; q < NSET; ++q) v += acc[i][q][c];
         accs[i][c] = v;
       }
-    stage0 += KT;
+    stage0 += KS;
 
     // ---- hand over and epilogue
     float* hw = handover + (rb * 32 + lane) * (4 * NT8);
@@ -370,8 +389,7 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
 
   // gate_up: W13 [E, 2I, H], activations x [T, H]
   p.blob = a.w13;
-  p.codes = reinterpret_cast<const uint32_t*>(a.w13 + blob_codes_offset());
-  p.scales = reinterpret_cast<const uint16_t*>(a.w13 + blob_scales_offset(a.E, 2 * a.I, a.H));
+  p.tiles = a.w13 + blob_tiles_offset();
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
@@ -383,8 +401,7 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
 
   // down: W2 [E, H, I], activations a [cap, I]
   p.blob = a.w2;
-  p.codes = reinterpret_cast<const uint32_t*>(a.w2 + blob_codes_offset());
-  p.scales = reinterpret_cast<const uint16_t*>(a.w2 + blob_scales_offset(a.E, a.H, a.I));
+  p.tiles = a.w2 + blob_tiles_offset();
   p.N = a.H;
   p.K = a.I;
   p.role = CHORD_ROLE_DOWN;

@@ -8,9 +8,14 @@
 // asynchronous by construction, so the overlap becomes warp specialisation:
 //
 //   warp 0      producer: per item (routing block b of up to 256 rows, 128-row weight
-//               tile nt) one bulk copy of the packed codes + scales per 128-wide K step
-//               into a raw ring, and the routed activation rows of each 64-wide K step
-//               gathered by TMA (tile::gather4, 128-byte swizzle) into the B ring.
+//               tile nt) one bulk copy of the packed codes + scales of two 128-wide K
+//               tiles into a raw ring, and per 64-wide K step the block's activation
+//               rows as tiled TMA boxes (64 and 16 rows, 128-byte swizzle) into the B
+//               ring. The rows are contiguous because the activations are in routing
+//               order: the intermediate of the down projection already is, and the
+//               gate_up input is permuted into that order first (a row gather by TMA
+//               moves 512 B per instruction and caps near 11 GB/s per SM; a 64-row box
+//               moves 8 KiB).
 //   warps 2..9  dequant: raw int4 -> bf16 (subtract 8, then scale) into the A ring in
 //               the UMMA K-major 128-byte-swizzle layout, 16 rows per warp.
 //   warp 1      MMA: one thread issues tcgen05.mma (M = 128 weight rows, N = the
@@ -32,7 +37,8 @@
 namespace chord {
 namespace {
 
-constexpr int kRawStages = 4;
+constexpr int kRawTiles = 2;   // 128-wide K tiles per raw stage (one bulk copy)
+constexpr int kRawStages = 3;
 constexpr int kAStages = 2;   // dequantised weights: produced on chip, double buffered
 constexpr int kBStages = 4;   // gathered activations: deep enough to cover TMA latency
 constexpr int kMaxN = 256;
@@ -43,12 +49,11 @@ constexpr int kTcThreads = 32 * (2 + kDequantWarps + kEpiWarps);
 
 constexpr int kAStageBytes = 128 * 64 * 2;
 constexpr int kBStageBytes = kMaxN * 64 * 2;
-constexpr int kRawStageBytes = kTileCodeBytes + kTileScaleBytes;
+constexpr int kRawStageBytes = kRawTiles * kTileBytes;
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kAStages * kAStageBytes;
 constexpr int kOffRaw = kOffB + kBStages * kBStageBytes;
-constexpr int kOffCoord = kOffRaw + kRawStages * kRawStageBytes;
-constexpr int kOffDesc = kOffCoord + kMaxN * 4;
+constexpr int kOffDesc = kOffRaw + kRawStages * kRawStageBytes;
 
 struct TcDesc {
   int e, nt, pos0, nvalid, end, pad[3];
@@ -61,8 +66,7 @@ constexpr int kTcSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the 
 enum Epi { kGateUp = 0, kDown = 1 };
 
 struct TcParams {
-  const uint8_t* codes;
-  const uint8_t* scales;
+  const uint8_t* tiles;
   const uint8_t* blob;
   int N, K, E, role;
   const int32_t* sorted_ids;
@@ -72,7 +76,6 @@ struct TcParams {
   int64_t n_slots;
   int topk;
   int64_t cap;
-  int act_rows;          // rows of the activation tensor map (out-of-range row = zero fill)
   uint16_t* a_out;
   float* y_out;
   const float* topk_weights;
@@ -84,6 +87,7 @@ struct TcParams {
 // rb*16 .. rb*16+15. Lane (g, t) converts the two words of K slices j = 2*hk, 2*hk+1 of
 // rows rb*16 + g and rb*16 + 8 + g; the slice order alternates with g so that the eight
 // lanes of each shared-memory phase hit eight distinct 16-byte bank groups.
+// `raw` addresses one 9216-byte tile (codes, then scales).
 __device__ __forceinline__ void dequant_half(uint32_t raw, uint32_t a_stage, int rb, int hk, int lane) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -102,9 +106,20 @@ __device__ __forceinline__ void dequant_half(uint32_t raw, uint32_t a_stage, int
   }
 }
 
+// TMA: tiled box of the activation tensor (64 columns x box rows), 128-byte swizzle.
+__device__ __forceinline__ void tma_tile2d(uint32_t dst, const void* tmap, int col, int row, uint64_t* bar,
+                                           uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(row), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act, TcParams p) {
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap64, const __grid_constant__ CUtensorMap tmap16,
+                   TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled operand stages
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -123,7 +138,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
   uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
-  int* coords = reinterpret_cast<int*>(smem + kOffCoord);
   TcDesc* descs = reinterpret_cast<TcDesc*>(smem + kOffDesc);
   __shared__ int abort_flag;
 
@@ -191,15 +205,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         pos0 = int(b * p.block_m);
         const bool e_ok = unsigned(e) < unsigned(p.E);
         for (int r = lane; r < kMaxN; r += 32) {
-          int coord = p.act_rows;     // out of range: reads as zero
           if (e_ok && r < p.block_m) {
             const int f = __ldg(p.sorted_ids + pos0 + r);
-            if (f >= 0 && f < p.n_slots) {
-              coord = (EPI == kGateUp) ? f / p.topk : pos0 + r;
-              nvalid = r + 1;
-            }
+            if (f >= 0 && f < p.n_slots) nvalid = r + 1;
           }
-          coords[r] = coord;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
@@ -222,7 +231,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       const int nmma = (nvalid + 15) & ~15;
       const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
-      for (int kt = 0; kt < KT && ok; ++kt) {
+      for (int kt0 = 0; kt0 < KT && ok; kt0 += kRawTiles) {
+        const int ntl = min(kRawTiles, KT - kt0);
         const uint32_t rs = rstage % kRawStages;
         if (rstage >= uint32_t(kRawStages) &&
             !mbar_wait(&raw_empty[rs], ((rstage / kRawStages) - 1) & 1, abort_v, p.status)) {
@@ -231,28 +241,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (lane == 0) {
           uint8_t* st = smem + kOffRaw + rs * kRawStageBytes;
-          mbar_arrive_expect_tx(&raw_full[rs], kRawStageBytes);
-          bulk_g2s_hint(st, p.codes + (tile0 + kt) * kTileCodeBytes, kTileCodeBytes, &raw_full[rs], pol_w);
-          bulk_g2s_hint(st + kTileCodeBytes, p.scales + (tile0 + kt) * kTileScaleBytes, kTileScaleBytes,
-                        &raw_full[rs], pol_w);
+          mbar_arrive_expect_tx(&raw_full[rs], uint32_t(ntl) * kTileBytes);
+          bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &raw_full[rs],
+                        pol_w);
         }
         ++rstage;
-        for (int hk = 0; hk < 2; ++hk) {
+        for (int sub = 0; sub < 2 * ntl; ++sub) {
           const uint32_t s = bstage % kBStages;
           if (bstage >= uint32_t(kBStages) &&
               !mbar_wait(&b_empty[s], ((bstage / kBStages) - 1) & 1, abort_v, p.status)) {
             ok = false;
             break;
           }
-          if (lane == 0) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
-          __syncwarp();
-          const uint32_t bst = sbase + kOffB + s * kBStageBytes;
-          const int col = kt * kTileK + hk * 64;
-          for (int i = lane; i < nmma / 4; i += 32)
-            tma_gather4(bst + i * 512, &tmap_act, col, coords[4 * i], coords[4 * i + 1],
-                        coords[4 * i + 2], coords[4 * i + 3], &b_full[s], pol_a);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
+            const uint32_t bst = sbase + kOffB + s * kBStageBytes;
+            const int col = kt0 * kTileK + sub * 64;
+            int r0 = 0;
+            for (; r0 + 64 <= nmma; r0 += 64) tma_tile2d(bst + r0 * 128, &tmap64, col, pos0 + r0, &b_full[s], pol_a);
+            for (; r0 < nmma; r0 += 16) tma_tile2d(bst + r0 * 128, &tmap16, col, pos0 + r0, &b_full[s], pol_a);
+          }
           ++bstage;
         }
+        __syncwarp();
       }
       __syncwarp();
     }
@@ -323,18 +334,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&dempty[ds]);
       if (end) break;
       bool ok = true;
-      for (int kt = 0; kt < KT && ok; ++kt) {
+      for (int kt0 = 0; kt0 < KT && ok; kt0 += kRawTiles) {
+        const int ntl = min(kRawTiles, KT - kt0);
         const uint32_t rs = rstage % kRawStages;
         if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
         const uint32_t raw = sbase + kOffRaw + rs * kRawStageBytes;
-        for (int hk = 0; hk < 2; ++hk) {
+        for (int sub = 0; sub < 2 * ntl; ++sub) {
           const uint32_t s = abstage % kAStages;
           if (abstage >= uint32_t(kAStages) &&
               !mbar_wait(&a_empty[s], ((abstage / kAStages) - 1) & 1, abort_v, p.status)) {
             ok = false;
             break;
           }
-          dequant_half(raw, sbase + kOffA + s * kAStageBytes, rb, hk, lane);
+          dequant_half(raw + (sub >> 1) * kTileBytes, sbase + kOffA + s * kAStageBytes, rb, sub & 1, lane);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
@@ -427,13 +439,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (row-major), box 64 columns x 1 row, 128-byte swizzle.
-cudaError_t make_row_gather_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
+// 2-D bf16 tensor [rows, cols] (row-major), box 64 columns x box_rows rows, 128-byte
+// swizzle; rows past the end read as zero.
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -441,12 +454,34 @@ cudaError_t make_row_gather_map(CUtensorMap* map, const void* base, int64_t rows
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// xs[pos, :] = x[sorted_ids[pos] / topk, :] for every routed position (16 B per thread).
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
+                                                           const int32_t* __restrict__ sorted_ids,
+                                                           const int32_t* __restrict__ ntp_p, int64_t cap,
+                                                           int64_t n_slots, int topk, int H,
+                                                           uint16_t* __restrict__ xs) {
+  int64_t ntp = *ntp_p;
+  if (ntp < 0) ntp = 0;
+  if (ntp > cap) ntp = cap;
+  const int vec = H / 8;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < ntp * vec;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t pos = i / vec;
+    const int c = int(i % vec) * 8;
+    const int f = __ldg(sorted_ids + pos);
+    if (f < 0 || f >= n_slots) continue;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + int64_t(f / topk) * H + c));
+    *reinterpret_cast<uint4*>(xs + pos * H + c) = v;
+  }
+}
+
 template <int EPI>
-cudaError_t launch_one(const CUtensorMap& map, const TcParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const TcParams& p, int grid,
+                       cudaStream_t stream) {
   auto kern = tc_gemm_kernel<EPI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kTcThreads, kTcSmemBytes, stream>>>(map, p);
+  kern<<<grid, kTcThreads, kTcSmemBytes, stream>>>(m64, m16, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -471,30 +506,38 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
   p.status = a.status;
   const int grid = a.num_sms;
 
-  // gate_up: W13 [E, 2I, H]; B rows gathered from x [T, H] by token
-  CUtensorMap map;
-  cudaError_t err = make_row_gather_map(&map, a.x, a.T, a.H);
+  // gate_up: W13 [E, 2I, H]; B rows from the hidden states permuted into routing order
+  {
+    const int64_t total = a.cap * (a.H / 8);
+    int64_t g = (total + 255) / 256;
+    if (g > int64_t(a.num_sms) * 16) g = int64_t(a.num_sms) * 16;
+    permute_rows_kernel<<<unsigned(g), 256, 0, stream>>>(a.x, a.sorted_ids, a.ntp, a.cap, a.T * a.topk, a.topk,
+                                                         a.H, a.xs);
+    count_launches(1);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+  }
+  CUtensorMap m64, m16;
+  cudaError_t err = make_tile_map(&m64, a.xs, a.cap, a.H, 64);
+  if (err == cudaSuccess) err = make_tile_map(&m16, a.xs, a.cap, a.H, 16);
   if (err != cudaSuccess) return err;
   p.blob = a.w13;
-  p.codes = a.w13 + blob_codes_offset();
-  p.scales = a.w13 + blob_scales_offset(a.E, 2 * a.I, a.H);
+  p.tiles = a.w13 + blob_tiles_offset();
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
-  p.act_rows = int(a.T);
-  if ((err = launch_one<kGateUp>(map, p, grid, stream)) != cudaSuccess) return err;
+  if ((err = launch_one<kGateUp>(m64, m16, p, grid, stream)) != cudaSuccess) return err;
   if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
 
-  // down: W2 [E, H, I]; B rows of the intermediate a [cap, I] by sorted position
-  if ((err = make_row_gather_map(&map, a.a, a.cap, a.I)) != cudaSuccess) return err;
+  // down: W2 [E, H, I]; B rows of the intermediate a [cap, I], already in routing order
+  if ((err = make_tile_map(&m64, a.a, a.cap, a.I, 64)) != cudaSuccess) return err;
+  if ((err = make_tile_map(&m16, a.a, a.cap, a.I, 16)) != cudaSuccess) return err;
   p.blob = a.w2;
-  p.codes = a.w2 + blob_codes_offset();
-  p.scales = a.w2 + blob_scales_offset(a.E, a.H, a.I);
+  p.tiles = a.w2 + blob_tiles_offset();
   p.N = a.H;
   p.K = a.I;
   p.role = CHORD_ROLE_DOWN;
-  p.act_rows = int(a.cap);
-  return launch_one<kDown>(map, p, grid, stream);
+  return launch_one<kDown>(m64, m16, p, grid, stream);
 }
 
 }  // namespace chord
