@@ -107,6 +107,27 @@ CHORD_API chord_status_t chord_moe_align(const int32_t* topk_ids /* device [T, t
                                int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
                                size_t workspace_bytes, chord_stream_t stream);
 
+/* Routing sort for callers that cannot allocate device memory (no counterpart on the
+ * pages). Same arguments, results and limits as chord_moe_align, minus the workspace:
+ * the scratch that large batches need lives in a static device array of 576 KiB that
+ * every GPU loading this library holds until the process exits. Made for callers that
+ * may not call cudaMalloc where they route a batch, e.g. a serving engine that reserved
+ * all free device memory up front, or code running under stream capture without a
+ * workspace tensor at hand.
+ *  - T*topk must be <= 131072 (2^17); larger batches return CHORD_ERR_UNSUPPORTED.
+ *  - Allocates nothing. The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device); make that first call before any stream
+ *    capture.
+ *  - All calls share the array. Nothing in it needs to start at zero (each call
+ *    overwrites every entry it later reads), but calls that overlap on the GPU (other
+ *    streams, other host threads) race on it: serialise them.
+ * Returns CHORD_ERR_INVALID_ARG for bad sizes or null pointers, CHORD_ERR_CUDA when the
+ * address lookup or a launch fails. */
+CHORD_API chord_status_t chord_moe_align_noalloc(const int32_t* topk_ids, int64_t T, int topk, int E,
+                                                 int block_m, int32_t* sorted_ids, int32_t* expert_ids,
+                                                 int32_t* num_tokens_padded, int32_t* expert_offsets,
+                                                 chord_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * One-time weight repack ("Gruppierte SM90-Kernel": prepared weights are permuted INT4
  * buffers with re-laid scales, and the mode is recorded in the prepared weight and

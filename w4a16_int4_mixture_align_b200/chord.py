@@ -53,6 +53,7 @@ SIGNATURES = {
     "chord_moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _I64, _I, _I, _I, _I, _P, _P,
                                _SZ, _I, _P]),
     "chord_moe_check_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "chord_moe_align_noalloc": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
 }
@@ -146,6 +147,17 @@ def chord_moe_align(topk_ids, E, block_m, sorted_ids, expert_ids, num_tokens_pad
     _check(lib().chord_moe_align(_ptr(topk_ids), T, topk, E, block_m, _ptr(sorted_ids),
                                  _ptr(expert_ids), _ptr(num_tokens_padded), _ptr(expert_offsets),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "chord_moe_align")
+
+
+def chord_moe_align_noalloc(topk_ids, E, block_m, sorted_ids, expert_ids, num_tokens_padded,
+                            expert_offsets=None, stream=None):
+    """chord_moe_align without a workspace: its scratch is a static device array in the
+    library (for callers that cannot allocate device memory when they route)."""
+    T, topk = topk_ids.shape
+    _check(lib().chord_moe_align_noalloc(_ptr(topk_ids), T, topk, E, block_m, _ptr(sorted_ids),
+                                         _ptr(expert_ids), _ptr(num_tokens_padded),
+                                         _ptr(expert_offsets), _stream(stream)),
+           "chord_moe_align_noalloc")
 
 
 def chord_repack_weights(qweight, scales, role, out, group_size=32, stream=None):
