@@ -144,6 +144,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread (up to `hint_ns`) until the phase completes,
+// instead of returning at once: waiting warps then cost no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of `bar` to complete. Returns false (and raises the CTA's
 // abort flag and the device status) when the wait gave up or another thread aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -151,7 +165,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -241,6 +255,13 @@ __device__ __forceinline__ void dequant8(uint32_t word, uint32_t s2, uint32_t ou
 }
 
 __device__ __forceinline__ uint32_t bf16_splat(uint16_t s) { return uint32_t(s) * 0x10001u; }
+
+// The low (hi = 0) or high (hi = 1) bf16 of `pair` in both halves (one byte permute).
+__device__ __forceinline__ uint32_t bf16_splat_half(uint32_t pair, int hi) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(pair), "r"(hi ? 0x3232u : 0x1010u));
+  return d;
+}
 
 // D (f32 16x8) += A (bf16 16x16, row) * B (bf16 16x8, col). Not volatile: a pure
 // function of its operands, so the compiler may interleave it with independent work.

@@ -10,8 +10,9 @@
 //                 it publishes a descriptor, then per stage of KTS consecutive 128-wide
 //                 K tiles issues ONE bulk copy of their codes + scales (up to 36 KiB:
 //                 a bulk copy has a high fixed cost, so bytes per copy decide the
-//                 streaming rate) and cp.async copies of the routed activation rows,
-//                 all completing on the stage's mbarrier.
+//                 streaming rate). The few routed activation rows are small and shared
+//                 by every warp, so consumers read them straight from global memory
+//                 through L1 (ld.global.nc) instead of staging them.
 //   warps 1..8    consumer group 0, warps 9..16 group 1: group g takes the tiles of
 //                 parity g inside each stage; warp w owns 16 physical rows. Codes go
 //                 shared -> registers and dequantise to bf16 pairs (subtract 8, then
@@ -62,10 +63,8 @@ struct ItemDesc {
 
 template <int TC>
 struct Smem {
-  static constexpr int kKTS = TC <= 16 ? 4 : 2;                 // K tiles per stage
-  static constexpr int kStageAct = kKTS * kTileBytes;           // activation rows after the tiles
-  static constexpr int kActPitch = kKTS * 256 + 64;             // padded row pitch (bank spread)
-  static constexpr int kStageBytes = ((kStageAct + TC * kActPitch) + 127) / 128 * 128;
+  static constexpr int kKTS = 4;                                // K tiles per stage
+  static constexpr int kStageBytes = kKTS * kTileBytes;
   static constexpr int kHandoverBytes = 8 * 32 * (TC / 8) * 4 * 4;  // 8 warps x 32 lanes x 4*NT floats
   static constexpr int kBudget = 200 * 1024;
   static constexpr int kFit =
@@ -75,12 +74,51 @@ struct Smem {
       kStages * kStageBytes + kHandoverBytes + kDescRing * int(sizeof(ItemDesc)) + 1024;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+__device__ __forceinline__ uint4 ldg_nc128(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
 }
-// Arrives on `bar` once this thread's earlier cp.async copies have landed.
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+
+// Dequantises NTILE tiles of a stage (tiles t0, t0 + 2, ...) for warp `rb` (16 rows) and
+// accumulates them against the routed activation rows (xrow[n8] points at this lane's row
+// of 8-token tile n8, advanced to the stage's first K): the A fragments of
+// mma.m16n8k16 come straight out of dequant8; tokens are the N dimension.
+template <int NT8, int NSET, int NTILE, class S>
+__device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb, int lane,
+                                              const uint16_t* const (&xrow)[NT8],
+                                              float (&acc)[NT8][NSET][4]) {
+  const int g = lane >> 2, t = lane & 3;
+  uint4 c0[NTILE], c1[NTILE], sv[NTILE];
+#pragma unroll
+  for (int u = 0; u < NTILE; ++u) {
+    const uint8_t* st = stg + (t0 + 2 * u) * kTileBytes;
+    c0[u] = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
+    c1[u] = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
+    sv[u] = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + g * 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int u = 0; u < NTILE; ++u) {
+      const uint32_t cw0 = j == 0 ? c0[u].x : j == 1 ? c0[u].y : j == 2 ? c0[u].z : c0[u].w;
+      const uint32_t cw1 = j == 0 ? c1[u].x : j == 1 ? c1[u].y : j == 2 ? c1[u].z : c1[u].w;
+      // scale pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
+      const uint32_t sp0 = (j >> 1) ? sv[u].y : sv[u].x;
+      const uint32_t sp1 = (j >> 1) ? sv[u].w : sv[u].z;
+      uint32_t w0[4], w1[4];
+      dequant8(cw0, bf16_splat_half(sp0, j & 1), w0);
+      dequant8(cw1, bf16_splat_half(sp1, j & 1), w1);
+      const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
+      const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8) {
+        const uint4 xv = ldg_nc128(xrow[n8] + (t0 + 2 * u) * kTileK + 32 * j + 8 * t);
+        mma_bf16_16816(acc[n8][(2 * u) % NSET], a_lo, xv.x, xv.y);
+        mma_bf16_16816(acc[n8][(2 * u + 1) % NSET], a_hi, xv.z, xv.w);
+      }
+    }
+  }
 }
 
 template <int EPI, int TC>
@@ -114,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       if (blockIdx.x == 0) atomicOr(p.status, CHORD_DEV_BLOB_MISMATCH);
     }
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1 + 32);  // producer expect_tx + one cp.async arrival per lane
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
     for (int s = 0; s < kDescRing; ++s) {
@@ -142,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     const int64_t nblocks = ntp / p.block_m;
     const int64_t items = nblocks * cpb * NTILES;
     const uint64_t pol_w = policy_evict_first();
-    const uint64_t pol_a = policy_evict_last();
     uint32_t stage = 0;      // global stage counter
     uint32_t nitem = 0;      // published descriptors
     for (int64_t w = blockIdx.x;; w += gridDim.x) {
@@ -177,10 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       if (lane == 0) mbar_arrive(&dfull[ds]);
       ++nitem;
       if (end) break;
-      // stream the item: one bulk copy of KTS tiles (codes + scales) per stage, and the
-      // routed activation rows by cp.async (16 B per lane per copy)
-      const int64_t act_row = (EPI == kGateUp) ? int64_t(fval / p.topk) : int64_t(pos0 + lane);
-      const uint16_t* act_src = p.act + act_row * p.act_ld;
+      // stream the item: one bulk copy of KTS tiles (codes + scales) per stage
       const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
       bool ok = true;
       for (int ks = 0; ks < KS; ++ks, ++stage) {
@@ -192,28 +226,16 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
         }
         const int kt0 = ks * KTS;
         const int ntl = min(KTS, KT - kt0);
-        uint8_t* st = stages + slot * S::kStageBytes;
         if (lane == 0) {
+          uint8_t* st = stages + slot * S::kStageBytes;
           mbar_arrive_expect_tx(&full[slot], uint32_t(ntl) * kTileBytes);
           bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &full[slot],
                         pol_w);
         }
-        const int chunks_per_row = ntl * 16;
-        const uint32_t act_base = smem_u32(st + S::kStageAct);
-        for (int c = lane; c < TC * 16 * KTS; c += 32) {
-          const int r = c / (16 * KTS), q = c % (16 * KTS);
-          const int f = __shfl_sync(0xffffffffu, fval, r);
-          const uint16_t* src = reinterpret_cast<const uint16_t*>(
-              __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(act_src), r));
-          if (f >= 0 && q < chunks_per_row)
-            cp_async16(act_base + r * S::kActPitch + q * 16, src + kt0 * kTileK + q * 8);
-        }
-        cp_async_arrive(&full[slot]);
       }
       if (!ok) break;
     }
     // drain: wait (bounded, ignoring the abort flag) for every copy still in flight
-    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       int dummy = 0;
       const uint32_t first = stage > uint32_t(NSTAGE) ? stage - NSTAGE : 0;
@@ -234,6 +256,15 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     if (!mbar_wait(&dfull[ds], (it / kDescRing) & 1, abort_v, p.status)) return;
     const ItemDesc& d = descs[ds];
     if (d.end) return;
+    // this lane's activation row of each 8-token tile (padding columns read row 0: their
+    // results are discarded by the epilogue)
+    const uint16_t* xrow0[NT8];
+#pragma unroll
+    for (int n8 = 0; n8 < NT8; ++n8) {
+      const int f = d.f[n8 * 8 + g];
+      const int64_t row = f < 0 ? 0 : ((EPI == kGateUp) ? int64_t(f / p.topk) : int64_t(d.pos0 + n8 * 8 + g));
+      xrow0[n8] = p.act + row * p.act_ld;
+    }
     // independent accumulator chains per 8-token tile so consecutive MMAs overlap
     constexpr int NSET = NT8 >= 4 ? 1 : (4 / NT8);
     float acc[NT8][NSET][4];
@@ -250,32 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       // plain shared loads (ordered after the wait by its memory clobber) so the compiler
       // can schedule them ahead of the dequantisation and the MMAs
       const uint8_t* stg = stages + slot * S::kStageBytes;
-      for (int i = grp; i < ntl; i += 2) {
-        const uint8_t* st = stg + i * kTileBytes;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
-        const uint4 sv = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + g * 16);
-        const uint8_t* act = stg + S::kStageAct + g * S::kActPitch + i * 256 + t * 16;
-        const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
-        const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};  // bf16 pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
+      const uint16_t* xrow[NT8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint16_t s0 = uint16_t(sw[j >> 1] >> (16 * (j & 1)));
-          const uint16_t s1 = uint16_t(sw[2 + (j >> 1)] >> (16 * (j & 1)));
-          uint32_t w0[4], w1[4];
-          dequant8(cw0[j], bf16_splat(s0), w0);
-          dequant8(cw1[j], bf16_splat(s1), w1);
-          const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
-          const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
-#pragma unroll
-          for (int n8 = 0; n8 < NT8; ++n8) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(act + n8 * 8 * S::kActPitch + j * 64);
-            mma_bf16_16816(acc[n8][j % NSET], a_lo, xv.x, xv.y);
-            mma_bf16_16816(acc[n8][(j + NSET / 2) % NSET], a_hi, xv.z, xv.w);
-          }
-        }
-      }
+      for (int n8 = 0; n8 < NT8; ++n8) xrow[n8] = xrow0[n8] + ks * KTS * kTileK;
+      for (int i = grp; i < ntl; i += 2) consume_tiles<NT8, NSET, 1, S>(stg, i, rb, lane, xrow, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }

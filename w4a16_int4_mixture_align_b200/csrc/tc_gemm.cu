@@ -83,23 +83,42 @@ struct TcParams {
   uint32_t* status;
 };
 
-// Dequantises half (64 K) of a raw 128x128 tile into an A stage: warp `rb` writes rows
-// rb*16 .. rb*16+15. Lane (g, t) converts the two words of K slices j = 2*hk, 2*hk+1 of
-// rows rb*16 + g and rb*16 + 8 + g; the slice order alternates with g so that the eight
-// lanes of each shared-memory phase hit eight distinct 16-byte bank groups.
-// `raw` addresses one 9216-byte tile (codes, then scales).
-__device__ __forceinline__ void dequant_half(uint32_t raw, uint32_t a_stage, int rb, int hk, int lane) {
+// Loads lane (g, t)'s share of one raw 128x128 tile (at `raw`: codes, then scales) for
+// warp `rb`: the 16-byte code vectors of rows rb*16 + g (h = 0) and rb*16 + 8 + g (h = 1),
+// each holding K slices j = 0..3 at 8t, and the matching 4 group scales per row. Each
+// quarter-warp reads 8 distinct 16-byte bank groups.
+struct TileShare {
+  uint4 c[2];
+  uint2 s[2];
+};
+__device__ __forceinline__ TileShare load_share(uint32_t raw, int rb, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  TileShare v;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    v.c[h] = lds128(raw + rb * 1024 + h * 512 + g * 64 + t * 16);
+    v.s[h] = lds64(raw + kTileCodeBytes + rb * 128 + g * 16 + h * 8);
+  }
+  return v;
+}
+
+// Dequantises half hk (64 K) of the tile share into an A stage (UMMA K-major, 128-byte
+// swizzle): slices j = 2*hk, 2*hk+1. The slice order alternates with g so that the
+// eight lanes of each 16-byte store phase hit eight distinct bank groups.
+template <int HK>
+__device__ __forceinline__ void dequant_half(const TileShare& v, uint32_t a_stage, int rb, int lane) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint2 w = lds64(raw + rb * 1024 + h * 512 + g * 64 + t * 16 + hk * 8);
-    const uint32_t s = lds32(raw + kTileCodeBytes + rb * 128 + g * 16 + h * 8 + hk * 4);
+    const uint32_t w0 = HK ? v.c[h].z : v.c[h].x;  // slice 2*HK
+    const uint32_t w1 = HK ? v.c[h].w : v.c[h].y;  // slice 2*HK + 1
+    const uint32_t sp = HK ? v.s[h].y : v.s[h].x;  // their two scales
     const int r = rb * 16 + 8 * h + g;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int jj = (q + g) & 1;
       uint32_t o[4];
-      dequant8(jj ? w.y : w.x, bf16_splat(uint16_t(jj ? (s >> 16) : (s & 0xFFFFu))), o);
+      dequant8(jj ? w1 : w0, bf16_splat_half(sp, jj), o);
       const int c = 4 * jj + t;
       sts128(a_stage + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4), o);
     }
@@ -339,14 +358,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t rs = rstage % kRawStages;
         if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
         const uint32_t raw = sbase + kOffRaw + rs * kRawStageBytes;
+        TileShare share;
         for (int sub = 0; sub < 2 * ntl; ++sub) {
+          if ((sub & 1) == 0) share = load_share(raw + (sub >> 1) * kTileBytes, rb, lane);
           const uint32_t s = abstage % kAStages;
           if (abstage >= uint32_t(kAStages) &&
               !mbar_wait(&a_empty[s], ((abstage / kAStages) - 1) & 1, abort_v, p.status)) {
             ok = false;
             break;
           }
-          dequant_half(raw + (sub >> 1) * kTileBytes, sbase + kOffA + s * kAStageBytes, rb, sub & 1, lane);
+          if (sub & 1)
+            dequant_half<1>(share, sbase + kOffA + s * kAStageBytes, rb, lane);
+          else
+            dequant_half<0>(share, sbase + kOffA + s * kAStageBytes, rb, lane);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
