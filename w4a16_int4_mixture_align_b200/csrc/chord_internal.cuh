@@ -127,6 +127,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -302,7 +305,7 @@ struct ForwardArgs {
   const uint8_t* w2;
   uint16_t* out;
   uint16_t* a;     // [cap, I] bf16 intermediate, indexed by sorted position
-  float* y;        // [T*topk, H] fp32 weighted expert outputs, indexed by flat slot
+  float* y;        // [T*topk, H] fp32 expert outputs (before the top-k weight), by flat slot
   uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
   uint32_t* status;
   int64_t T;

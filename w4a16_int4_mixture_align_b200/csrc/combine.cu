@@ -1,8 +1,9 @@
 // combine.cu -- top-k weighted combine and optional routing validation.
 //
-// The down kernels write y[f, :] = topk_weights[f] * (W2[e] . a) for every local flat
-// slot f. The combine sums those rows over a token's local slots in ascending slot
-// order in FP32 and rounds once to BF16; a token with no local slot gets a zero row.
+// The down kernels write y[f, :] = W2[e] . a for every local flat slot f. The combine
+// multiplies each row by its top-k weight and sums over the token's local slots in
+// ascending slot order in FP32 (acc += w_j * y_j), then rounds once to BF16; a token with
+// no local slot gets a zero row.
 // The blog excludes this step from its kernel timings ("Messungen"); here it is one
 // HBM-bound pass reading T*topk_local*H*4 bytes and writing T*H*2 bytes.
 #include "chord_internal.cuh"
@@ -12,6 +13,7 @@ namespace {
 
 // One thread per 8 consecutive outputs of one token.
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ topk_ids,
+                                                      const float* __restrict__ topk_weights,
                                                       const float* __restrict__ y,
                                                       uint16_t* __restrict__ out, int64_t T,
                                                       int H, int topk, int E) {
@@ -25,10 +27,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
     for (int j = 0; j < topk; ++j) {
       const int e = __ldg(topk_ids + t * topk + j);
       if (unsigned(e) >= unsigned(E)) continue;
+      const float w = __ldg(topk_weights + t * topk + j);
       const float4* src = reinterpret_cast<const float4*>(y + (t * topk + j) * int64_t(H) + c);
       const float4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
-      acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
-      acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+      // product rounded, then added (no fused multiply-add), as the layer is defined
+      acc[0] = __fadd_rn(acc[0], __fmul_rn(w, v0.x)); acc[1] = __fadd_rn(acc[1], __fmul_rn(w, v0.y));
+      acc[2] = __fadd_rn(acc[2], __fmul_rn(w, v0.z)); acc[3] = __fadd_rn(acc[3], __fmul_rn(w, v0.w));
+      acc[4] = __fadd_rn(acc[4], __fmul_rn(w, v1.x)); acc[5] = __fadd_rn(acc[5], __fmul_rn(w, v1.y));
+      acc[6] = __fadd_rn(acc[6], __fmul_rn(w, v1.z)); acc[7] = __fadd_rn(acc[7], __fmul_rn(w, v1.w));
     }
     uint4 o;
     o.x = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[0]))) |
@@ -76,7 +82,8 @@ cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (total == 0) return cudaSuccess;
   int64_t grid = (total + 255) / 256;
   if (grid > int64_t(a.num_sms) * 16) grid = int64_t(a.num_sms) * 16;
-  combine_kernel<<<unsigned(grid), 256, 0, stream>>>(a.topk_ids, a.y, a.out, a.T, a.H, a.topk, a.E);
+  combine_kernel<<<unsigned(grid), 256, 0, stream>>>(a.topk_ids, a.topk_weights, a.y, a.out, a.T, a.H,
+                                                      a.topk, a.E);
   count_launches(1);
   return cudaGetLastError();
 }

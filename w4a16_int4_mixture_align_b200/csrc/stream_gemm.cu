@@ -19,7 +19,8 @@
 //                 scale) that are exactly the A fragments of mma.m16n8k16; tokens are N.
 //   epilogue      group 1 hands its partial sums to group 0, which adds them and applies
 //                 SiLU(gate)*up (gate_up; gate and up rows are interleaved by the repack)
-//                 or the top-k weight (down, written to the per-slot buffer y).
+//                 or writes the expert output (down) to the per-slot buffer y, which the
+//                 combine weights and sums.
 //
 // Every wait is an mbarrier wait bounded in time; on timeout the CTA raises
 // CHORD_DEV_TIMEOUT, unwinds, and the producer waits (bounded) for its copies in flight.
@@ -182,22 +183,39 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     const uint64_t pol_w = policy_evict_first();
     uint32_t stage = 0;      // global stage counter
     uint32_t nitem = 0;      // published descriptors
+    // routing metadata of item w: its expert and this lane's flat slot (lane < TC). The
+    // loads run kLook items ahead (a small register queue) so their latency overlaps
+    // the streaming of earlier items instead of stalling at every item boundary.
+    constexpr int kLook = 4;
+    auto load_meta = [&](int64_t w, int& e, int& pos0, int& f) {
+      e = -1;
+      pos0 = 0;
+      f = -1;
+      if (w >= items) return;
+      const int64_t bc = w / NTILES;
+      const int64_t b = bc / cpb;
+      const int c = int(bc % cpb);
+      e = __ldg(p.expert_ids + b);
+      pos0 = int(b * p.block_m) + c * TC;
+      const int lim = int(b * p.block_m) + p.block_m;
+      if (lane < TC && pos0 + lane < lim) f = __ldg(p.sorted_ids + pos0 + lane);
+    };
+    int qe[kLook], qpos[kLook], qf[kLook];
+#pragma unroll
+    for (int i = 0; i < kLook; ++i) load_meta(blockIdx.x + int64_t(i) * gridDim.x, qe[i], qpos[i], qf[i]);
     for (int64_t w = blockIdx.x;; w += gridDim.x) {
       const bool end = w >= items;
-      int e = -1, nt = 0, pos0 = 0, fval = -1;
+      int e = qe[0], pos0 = qpos[0], fval = qf[0];
+      const int nt = end ? 0 : int(w % NTILES);
+#pragma unroll
+      for (int i = 0; i + 1 < kLook; ++i) {
+        qe[i] = qe[i + 1];
+        qpos[i] = qpos[i + 1];
+        qf[i] = qf[i + 1];
+      }
+      load_meta(w + int64_t(kLook) * gridDim.x, qe[kLook - 1], qpos[kLook - 1], qf[kLook - 1]);
       if (!end) {
-        nt = int(w % NTILES);
-        const int64_t bc = w / NTILES;
-        const int64_t b = bc / cpb;
-        const int c = int(bc % cpb);
-        e = __ldg(p.expert_ids + b);
-        pos0 = int(b * p.block_m) + c * TC;
-        const int lim = int(b * p.block_m) + p.block_m;
-        if (lane < TC && pos0 + lane < lim) {
-          const int f = __ldg(p.sorted_ids + pos0 + lane);
-          if (f >= 0 && f < p.n_slots) fval = f;
-        }
-        if (unsigned(e) >= unsigned(p.E)) fval = -1;
+        if (!(fval >= 0 && fval < p.n_slots) || unsigned(e) >= unsigned(p.E)) fval = -1;
         if (__ballot_sync(0xffffffffu, fval >= 0) == 0) continue;  // nothing routed here
       }
       // publish the item (or the end marker) to the consumers
@@ -342,10 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
           const int col = n8 * 8 + 2 * t + q;
           const int f = d.f[col];
           if (f >= 0) {
-            const float wgt = __ldg(p.topk_weights + f);
             float* yr = p.y_out + int64_t(f) * p.H;
-            yr[n0] = accs[n8][q] * wgt;
-            yr[n0 + 8] = accs[n8][2 + q] * wgt;
+            yr[n0] = accs[n8][q];
+            yr[n0 + 8] = accs[n8][2 + q];
           }
         }
       }

@@ -23,8 +23,9 @@
 //               of two TMEM accumulators of 256 columns, and tcgen05.commit frees the
 //               ring stages and publishes the accumulator.
 //   warps 10..13 epilogue: tcgen05.ld of the accumulator; SiLU(gate)*up written to the
-//               bf16 intermediate (gate_up), or x topk_weight written to the per-slot
-//               fp32 buffer (down). Double buffering lets it overlap the next item.
+//               bf16 intermediate (gate_up), or the expert output written to the per-slot
+//               fp32 buffer (down; the combine applies the top-k weight). Double
+//               buffering lets it overlap the next item.
 //
 // Operand orientation follows the blog's decode profile (dequantised weights in the
 // MMA-M slot, tokens in N): one dequantised weight tile serves every token of a block.
@@ -214,20 +215,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint64_t pol_a = policy_evict_last();
     uint32_t rstage = 0, bstage = 0, nitem = 0;
     bool ok = true;
+    // routing metadata of item w (its expert and the flat slots of this lane's 8 rows),
+    // loaded one item ahead so the latency overlaps the current item's streaming
+    auto load_meta = [&](int64_t w, int& e, int (&f)[kMaxN / 32]) {
+      e = -1;
+#pragma unroll
+      for (int i = 0; i < kMaxN / 32; ++i) f[i] = -1;
+      if (w >= items) return;
+      const int64_t b = w / NTILES;
+      e = __ldg(p.expert_ids + b);
+      const int pos0 = int(b * p.block_m);
+#pragma unroll
+      for (int i = 0; i < kMaxN / 32; ++i) {
+        const int r = lane + 32 * i;
+        if (r < p.block_m) f[i] = __ldg(p.sorted_ids + pos0 + r);
+      }
+    };
+    int e_next, f_next[kMaxN / 32];
+    load_meta(blockIdx.x, e_next, f_next);
     for (int64_t w = blockIdx.x; ok; w += gridDim.x) {
       const bool end = w >= items;
-      int e = -1, nt = 0, pos0 = 0, nvalid = 0;
+      int e = e_next, nt = 0, pos0 = 0, nvalid = 0;
+      int fcur[kMaxN / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxN / 32; ++i) fcur[i] = f_next[i];
+      load_meta(w + gridDim.x, e_next, f_next);
       if (!end) {
         nt = int(w % NTILES);
-        const int64_t b = w / NTILES;
-        e = __ldg(p.expert_ids + b);
-        pos0 = int(b * p.block_m);
-        const bool e_ok = unsigned(e) < unsigned(p.E);
-        for (int r = lane; r < kMaxN; r += 32) {
-          if (e_ok && r < p.block_m) {
-            const int f = __ldg(p.sorted_ids + pos0 + r);
-            if (f >= 0 && f < p.n_slots) nvalid = r + 1;
-          }
+        pos0 = int((w / NTILES) * p.block_m);
+        if (unsigned(e) < unsigned(p.E)) {
+#pragma unroll
+          for (int i = 0; i < kMaxN / 32; ++i)
+            if (fcur[i] >= 0 && fcur[i] < p.n_slots) nvalid = lane + 32 * i + 1;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
@@ -394,28 +413,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&dempty[ds]);
       if (d.end) break;
       const uint32_t buf = it & 1;
+      // this item's flat slots, one per column, loaded before the accumulator wait so the
+      // global-load latency hides under the mainloop
+      int f_col[kMaxN / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxN / 32; ++i) {
+        const int c = lane + 32 * i;
+        f_col[i] = -1;
+        if (c < d.nvalid) {
+          const int f = __ldg(p.sorted_ids + d.pos0 + c);
+          if (f >= 0 && f < p.n_slots) f_col[i] = f;
+        }
+      }
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_v, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * 256;
-      for (int c0 = 0; c0 < d.nvalid; c0 += 16) {
+#pragma unroll
+      for (int cc = 0; cc < kMaxN / 16; ++cc) {
+        const int c0 = cc * 16;
+        if (c0 >= d.nvalid) break;
         float v[16];
         tmem_ld16(taddr + c0, v);
-        int f_l = -1;
-        float w_l = 0.f;
-        if (lane < 16 && c0 + lane < d.nvalid) {
-          const int f = __ldg(p.sorted_ids + d.pos0 + c0 + lane);
-          if (f >= 0 && f < p.n_slots) {
-            f_l = f;
-            if (EPI == kDown) w_l = __ldg(p.topk_weights + f);
-          }
-        }
+        // column c0 + c lives in lane (c0 + c) % 32 of register set (c0 + c) / 32
+        const int src_set = c0 >> 5;
+        int f_set = f_col[0];
+#pragma unroll
+        for (int i = 1; i < kMaxN / 32; ++i)
+          if (src_set == i) f_set = f_col[i];
         if (EPI == kGateUp) {
           const bool gate = (r & 15) < 8;
           const int i_col = d.nt * (kTileN / 2) + (r >> 4) * 8 + (r & 7);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
-            const int f = __shfl_sync(0xffffffffu, f_l, c);
+            const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
             if (gate && f >= 0)
               p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
                   __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
@@ -424,9 +455,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int n = d.nt * kTileN + r;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const int f = __shfl_sync(0xffffffffu, f_l, c);
-            const float wgt = __shfl_sync(0xffffffffu, w_l, c);
-            if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c] * wgt;
+            const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
+            if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c];
           }
         }
       }
