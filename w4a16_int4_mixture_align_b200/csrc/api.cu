@@ -213,7 +213,13 @@ int chord_select_block_m(int64_t T, int topk, int E_local, int E_global, int H, 
   if (tok_e <= 4.0) bm = 8;
   else if (tok_e <= 10.0) bm = 16;
   else if (tok_e <= 24.0) bm = 32;
-  else bm = 256;  // tensor-core schedule: one block per expert (up to 256 rows)
+  else {
+    // tensor-core schedule: one block should hold an expert's rows (the MMA N of an item
+    // is its routed rows rounded to 16, so spare capacity costs no MMA work), sized to the
+    // expected busiest expert (~1.5x the mean) so the activation ring stages stay small
+    const int want = int(tok_e * 1.5 + 15.0) / 16 * 16;
+    bm = want < 64 ? 64 : (want > 256 ? 256 : want);
+  }
   std::lock_guard<std::mutex> lk(g_mu);
   g_select_cache[key] = bm;
   return bm;

@@ -22,10 +22,15 @@
 //               block's routed rows rounded up to 16, K = 16 per instruction) into one
 //               of two TMEM accumulators of 256 columns, and tcgen05.commit frees the
 //               ring stages and publishes the accumulator.
-//   warps 10..13 epilogue: tcgen05.ld of the accumulator; SiLU(gate)*up written to the
-//               bf16 intermediate (gate_up), or the expert output written to the per-slot
+//   warps 10..17 epilogue (two per TMEM lane quadrant, alternate 16-column chunks):
+//               tcgen05.ld of the accumulator; SiLU(gate)*up written to the bf16
+//               intermediate (gate_up), or the expert output written to the per-slot
 //               fp32 buffer (down; the combine applies the top-k weight). Double
 //               buffering lets it overlap the next item.
+//
+// The rings are sized at launch from the largest MMA N of the call: a B stage holds N
+// rows, and the shared memory a small N leaves free becomes a deeper A ring, so the
+// dequant warps can run further ahead of the MMA.
 //
 // Operand orientation follows the blog's decode profile (dequantised weights in the
 // MMA-M slot, tokens in N): one dequantised weight tile serves every token of a block.
@@ -38,33 +43,66 @@
 namespace chord {
 namespace {
 
-constexpr int kRawTiles = 2;   // 128-wide K tiles per raw stage (one bulk copy)
+constexpr int kRawTiles = 2;      // 128-wide K tiles per raw stage (one bulk copy)
 constexpr int kRawStages = 3;
-constexpr int kAStages = 2;   // dequantised weights: produced on chip, double buffered
-constexpr int kBStages = 4;   // gathered activations: deep enough to cover TMA latency
+constexpr int kMaxStages = 8;     // upper bound of the A and B rings (runtime sized)
 constexpr int kMaxN = 256;
 constexpr int kDescRingTC = 8;
 constexpr int kDequantWarps = 8;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = 32 * (2 + kDequantWarps + kEpiWarps);
 
 constexpr int kAStageBytes = 128 * 64 * 2;
-constexpr int kBStageBytes = kMaxN * 64 * 2;
 constexpr int kRawStageBytes = kRawTiles * kTileBytes;
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kAStages * kAStageBytes;
-constexpr int kOffRaw = kOffB + kBStages * kBStageBytes;
-constexpr int kOffDesc = kOffRaw + kRawStages * kRawStageBytes;
 
 struct TcDesc {
   int e, nt, pos0, nvalid, end, pad[3];
 };
+// fixed part (from the 1024-aligned base): descriptors, barriers, TMEM slot; then rings
+constexpr int kOffDesc = 0;
 constexpr int kOffBar = kOffDesc + kDescRingTC * int(sizeof(TcDesc));
-constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 4 + 2 * kDescRingTC;
+constexpr int kNumBars = 2 * kRawStages + 4 * kMaxStages + 4 + 2 * kDescRingTC;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kTcSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack to align the base to 1024
+constexpr int kOffRings = 1024;
+static_assert(kOffTmemSlot + 16 <= kOffRings, "fixed part");
+constexpr int kSmemLimit = 232448 - 1024;  // 227 KiB opt-in per CTA, minus static shared
+
+// Ring geometry for a launch whose largest MMA N is nmax.
+struct TcRings {
+  int a_stages, b_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
+};
+__host__ __device__ inline TcRings tc_rings(int nmax) {
+  TcRings r;
+  r.b_stage_bytes = nmax * 128;
+  const int avail = kSmemLimit - 1024 - kOffRings - kRawStages * kRawStageBytes;
+  // the activation ring covers TMA latency, so it gets every stage that fits next to a
+  // double-buffered A ring; what a small N leaves over deepens the A ring
+  int bs = (avail - 2 * kAStageBytes) / r.b_stage_bytes;
+  bs = bs < 2 ? 2 : (bs > kMaxStages ? kMaxStages : bs);
+  int as = (avail - bs * r.b_stage_bytes) / kAStageBytes;
+  as = as < 2 ? 2 : (as > kMaxStages ? kMaxStages : as);
+  r.a_stages = as;
+  r.b_stages = bs;
+  r.off_a = kOffRings;
+  r.off_b = r.off_a + as * kAStageBytes;
+  r.off_raw = r.off_b + bs * r.b_stage_bytes;
+  r.smem_bytes = r.off_raw + kRawStages * kRawStageBytes + 1024;  // + base alignment slack
+  return r;
+}
 
 enum Epi { kGateUp = 0, kDown = 1 };
+
+// Position in a ring of runtime size: slot index and the phase parity of its barriers.
+struct RingPos {
+  uint32_t slot = 0, phase = 0, count = 0;
+  __device__ __forceinline__ void next(uint32_t stages) {
+    ++count;
+    if (++slot == stages) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
 
 struct TcParams {
   const uint8_t* tiles;
@@ -82,47 +120,26 @@ struct TcParams {
   const float* topk_weights;
   int I, H;
   uint32_t* status;
+  TcRings rings;
 };
 
-// Loads lane (g, t)'s share of one raw 128x128 tile (at `raw`: codes, then scales) for
-// warp `rb`: the 16-byte code vectors of rows rb*16 + g (h = 0) and rb*16 + 8 + g (h = 1),
-// each holding K slices j = 0..3 at 8t, and the matching 4 group scales per row. Each
-// quarter-warp reads 8 distinct 16-byte bank groups.
-struct TileShare {
-  uint4 c[2];
-  uint2 s[2];
-};
-__device__ __forceinline__ TileShare load_share(uint32_t raw, int rb, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  TileShare v;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    v.c[h] = lds128(raw + rb * 1024 + h * 512 + g * 64 + t * 16);
-    v.s[h] = lds64(raw + kTileCodeBytes + rb * 128 + g * 16 + h * 8);
-  }
-  return v;
-}
-
-// Dequantises half hk (64 K) of the tile share into an A stage (UMMA K-major, 128-byte
-// swizzle): slices j = 2*hk, 2*hk+1. The slice order alternates with g so that the
-// eight lanes of each 16-byte store phase hit eight distinct bank groups.
+// Dequantises half hk (64 K) of one row's 128-K share into an A stage (UMMA K-major,
+// 128-byte swizzle). Lane (g, t) of dequant warp (rb, h) owns row r = rb*16 + 8h + g:
+// `c` holds its four code words (K slices j = 0..3 at offset 8t), `sp` the two scales
+// of slices 2hk, 2hk+1. The slice order alternates with g so the eight lanes of each
+// 16-byte store phase hit eight distinct bank groups.
 template <int HK>
-__device__ __forceinline__ void dequant_half(const TileShare& v, uint32_t a_stage, int rb, int lane) {
-  const int g = lane >> 2, t = lane & 3;
+__device__ __forceinline__ void dequant_row_half(const uint4& c, uint32_t sp, uint32_t a_stage, int r,
+                                                 int g, int t) {
+  const uint32_t w0 = HK ? c.z : c.x;
+  const uint32_t w1 = HK ? c.w : c.y;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t w0 = HK ? v.c[h].z : v.c[h].x;  // slice 2*HK
-    const uint32_t w1 = HK ? v.c[h].w : v.c[h].y;  // slice 2*HK + 1
-    const uint32_t sp = HK ? v.s[h].y : v.s[h].x;  // their two scales
-    const int r = rb * 16 + 8 * h + g;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int jj = (q + g) & 1;
-      uint32_t o[4];
-      dequant8(jj ? w1 : w0, bf16_splat_half(sp, jj), o);
-      const int c = 4 * jj + t;
-      sts128(a_stage + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4), o);
-    }
+  for (int q = 0; q < 2; ++q) {
+    const int jj = (q + g) & 1;
+    uint32_t o[4];
+    dequant8(jj ? w1 : w0, bf16_splat_half(sp, jj), o);
+    const int ch = 4 * jj + t;
+    sts128(a_stage + (r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4), o);
   }
 }
 
@@ -145,15 +162,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
+  const int AS = p.rings.a_stages, BS = p.rings.b_stages;
+  const int b_stage_bytes = p.rings.b_stage_bytes;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + kRawStages;
   uint64_t* a_full = raw_empty + kRawStages;
-  uint64_t* a_empty = a_full + kAStages;
-  uint64_t* b_full = a_empty + kAStages;
-  uint64_t* b_empty = b_full + kBStages;
-  uint64_t* acc_full = b_empty + kBStages;       // [2]
+  uint64_t* a_empty = a_full + kMaxStages;
+  uint64_t* b_full = a_empty + kMaxStages;
+  uint64_t* b_empty = b_full + kMaxStages;
+  uint64_t* acc_full = b_empty + kMaxStages;     // [2]
   uint64_t* acc_empty = acc_full + 2;            // [2]
   uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
   uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
@@ -174,11 +193,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kDequantWarps);
     }
-    for (int s = 0; s < kAStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&a_full[s], kDequantWarps);
       mbar_init(&a_empty[s], 1);
-    }
-    for (int s = 0; s < kBStages; ++s) {
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
@@ -213,7 +230,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t items = nblocks * NTILES;
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
-    uint32_t rstage = 0, bstage = 0, nitem = 0;
+    uint32_t rstage = 0, nitem = 0;
+    RingPos bpos;
     bool ok = true;
     // routing metadata of item w (its expert and the flat slots of this lane's 8 rows),
     // loaded one item ahead so the latency overlaps the current item's streaming
@@ -278,28 +296,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         if (lane == 0) {
-          uint8_t* st = smem + kOffRaw + rs * kRawStageBytes;
+          uint8_t* st = smem + p.rings.off_raw + rs * kRawStageBytes;
           mbar_arrive_expect_tx(&raw_full[rs], uint32_t(ntl) * kTileBytes);
           bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &raw_full[rs],
                         pol_w);
         }
         ++rstage;
         for (int sub = 0; sub < 2 * ntl; ++sub) {
-          const uint32_t s = bstage % kBStages;
-          if (bstage >= uint32_t(kBStages) &&
-              !mbar_wait(&b_empty[s], ((bstage / kBStages) - 1) & 1, abort_v, p.status)) {
+          const uint32_t s = bpos.slot;
+          // the slot's previous fill (one lap ago, opposite phase) must have been consumed
+          if (bpos.count >= uint32_t(BS) && !mbar_wait(&b_empty[s], bpos.phase ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
           }
           if (lane == 0) {
             mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
-            const uint32_t bst = sbase + kOffB + s * kBStageBytes;
+            const uint32_t bst = sbase + p.rings.off_b + s * b_stage_bytes;
             const int col = kt0 * kTileK + sub * 64;
             int r0 = 0;
             for (; r0 + 64 <= nmma; r0 += 64) tma_tile2d(bst + r0 * 128, &tmap64, col, pos0 + r0, &b_full[s], pol_a);
             for (; r0 < nmma; r0 += 16) tma_tile2d(bst + r0 * 128, &tmap16, col, pos0 + r0, &b_full[s], pol_a);
           }
-          ++bstage;
+          bpos.next(BS);
         }
         __syncwarp();
       }
@@ -310,13 +328,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int dummy = 0;
       for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
         mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
-      for (uint32_t s = (bstage > uint32_t(kBStages) ? bstage - kBStages : 0); s < bstage; ++s)
-        mbar_wait(&b_full[s % kBStages], (s / kBStages) & 1, &dummy, p.status);
+      // the last min(BS, fills) fills of the B ring, walking back from the current slot
+      RingPos back = bpos;
+      const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
+      for (uint32_t i = 0; i < n_back; ++i) {
+        if (back.slot == 0) {
+          back.slot = BS - 1;
+          back.phase ^= 1u;
+        } else {
+          --back.slot;
+        }
+        mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
+      }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t abstage = 0;
+      RingPos apos, bpos;
       uint64_t* last_bar = nullptr;
       uint32_t last_parity = 0;
       for (uint32_t it = 0;; ++it) {
@@ -332,15 +360,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t idesc = idesc_bf16_m128((d.nvalid + 15) & ~15);
         bool ok = true;
         for (int ks = 0; ks < 2 * KT; ++ks) {
-          const uint32_t sa = abstage % kAStages, pa = (abstage / kAStages) & 1;
-          const uint32_t sb = abstage % kBStages, pb = (abstage / kBStages) & 1;
+          const uint32_t sa = apos.slot, pa = apos.phase;
+          const uint32_t sb = bpos.slot, pb = bpos.phase;
           if (!mbar_wait(&a_full[sa], pa, abort_v, p.status) || !mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = sbase + kOffA + sa * kAStageBytes;
-          const uint32_t b_addr = sbase + kOffB + sb * kBStageBytes;
+          const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
+          const uint32_t b_addr = sbase + p.rings.off_b + sb * b_stage_bytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
@@ -349,7 +377,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_commit(&b_empty[sb]);
           last_bar = &b_empty[sb];
           last_parity = pb;
-          ++abstage;
+          apos.next(AS);
+          bpos.next(BS);
         }
         if (!ok) break;
         tc_commit(&acc_full[buf]);
@@ -363,7 +392,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp < 2 + kDequantWarps) {
     // ----------------------------------------------------------------- dequant
     const int rb = warp - 2;
-    uint32_t rstage = 0, abstage = 0;
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t rstage = 0;
+    RingPos apos;
     for (uint32_t it = 0;; ++it) {
       const uint32_t ds = it % kDescRingTC;
       if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
@@ -376,24 +407,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ntl = min(kRawTiles, KT - kt0);
         const uint32_t rs = rstage % kRawStages;
         if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
-        const uint32_t raw = sbase + kOffRaw + rs * kRawStageBytes;
-        TileShare share;
+        const uint32_t raw = sbase + p.rings.off_raw + rs * kRawStageBytes;
+        uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+        uint2 s0 = make_uint2(0, 0), s1 = s0;
         for (int sub = 0; sub < 2 * ntl; ++sub) {
-          if ((sub & 1) == 0) share = load_share(raw + (sub >> 1) * kTileBytes, rb, lane);
-          const uint32_t s = abstage % kAStages;
-          if (abstage >= uint32_t(kAStages) &&
-              !mbar_wait(&a_empty[s], ((abstage / kAStages) - 1) & 1, abort_v, p.status)) {
+          if ((sub & 1) == 0) {  // this lane's share of the next tile: rows rb*16+g and +8
+            const uint32_t tb = raw + (sub >> 1) * kTileBytes;
+            c0 = lds128(tb + rb * 1024 + g * 64 + t * 16);
+            c1 = lds128(tb + rb * 1024 + 512 + g * 64 + t * 16);
+            s0 = lds64(tb + kTileCodeBytes + rb * 128 + g * 16);
+            s1 = lds64(tb + kTileCodeBytes + rb * 128 + g * 16 + 8);
+          }
+          const uint32_t s = apos.slot;
+          if (apos.count >= uint32_t(AS) && !mbar_wait(&a_empty[s], apos.phase ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
           }
-          if (sub & 1)
-            dequant_half<1>(share, sbase + kOffA + s * kAStageBytes, rb, lane);
-          else
-            dequant_half<0>(share, sbase + kOffA + s * kAStageBytes, rb, lane);
+          const uint32_t a_stage = sbase + p.rings.off_a + s * kAStageBytes;
+          if (sub & 1) {
+            dequant_row_half<1>(c0, s0.y, a_stage, rb * 16 + g, g, t);
+            dequant_row_half<1>(c1, s1.y, a_stage, rb * 16 + 8 + g, g, t);
+          } else {
+            dequant_row_half<0>(c0, s0.x, a_stage, rb * 16 + g, g, t);
+            dequant_row_half<0>(c1, s1.x, a_stage, rb * 16 + 8 + g, g, t);
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
-          ++abstage;
+          apos.next(AS);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&raw_empty[rs]);
@@ -403,7 +444,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ----------------------------------------------------------------- epilogue
-    const int q = warp & 3;   // TMEM lane quadrant this warp may access
+    const int q = warp & 3;                        // TMEM lane quadrant this warp may access
+    const int half = (warp - 2 - kDequantWarps) >> 2;  // which 16-column chunks (even / odd)
     const int r = q * 32 + lane;
     for (uint32_t it = 0;; ++it) {
       const uint32_t ds = it % kDescRingTC;
@@ -432,6 +474,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int cc = 0; cc < kMaxN / 16; ++cc) {
         const int c0 = cc * 16;
         if (c0 >= d.nvalid) break;
+        if ((cc & 1) != half) continue;
         float v[16];
         tmem_ld16(taddr + c0, v);
         // column c0 + c lives in lane (c0 + c) % 32 of register set (c0 + c) / 32
@@ -533,9 +576,9 @@ template <int EPI>
 cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const TcParams& p, int grid,
                        cudaStream_t stream) {
   auto kern = tc_gemm_kernel<EPI>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kTcThreads, kTcSmemBytes, stream>>>(m64, m16, p);
+  kern<<<grid, kTcThreads, p.rings.smem_bytes, stream>>>(m64, m16, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -558,6 +601,7 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
   p.H = a.H;
   p.E = a.E;
   p.status = a.status;
+  p.rings = tc_rings(min(kMaxN, (a.block_m + 15) & ~15));
   const int grid = a.num_sms;
 
   // gate_up: W13 [E, 2I, H]; B rows from the hidden states permuted into routing order
