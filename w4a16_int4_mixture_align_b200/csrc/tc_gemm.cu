@@ -5,38 +5,50 @@
 // as possible. The Chord blog's H200 prefill kernels overlap the dequantisation of the
 // next K slice with the in-flight WGMMA group ("H200 Prefill und TP8": batched wait<1>
 // pipelining) and size block_m from the tokens routed per expert. On sm_100a the MMA is
-// asynchronous by construction, so the overlap becomes warp specialisation:
+// asynchronous by construction, so the overlap becomes warp specialisation, and the
+// kernel runs on CTA pairs (clusters of two, tcgen05 cta_group::2):
 //
-//   warp 0      producer: per item (routing block b of up to 256 rows, 128-row weight
-//               tile nt) one bulk copy of the packed codes + scales of two 128-wide K
-//               tiles into a raw ring, and per 64-wide K step the block's activation
-//               rows as tiled TMA boxes (64 and 16 rows, 128-byte swizzle) into the B
-//               ring. The rows are contiguous because the activations are in routing
-//               order: the intermediate of the down projection already is, and the
-//               gate_up input is permuted into that order first (a row gather by TMA
-//               moves 512 B per instruction and caps near 11 GB/s per SM; a 64-row box
-//               moves 8 KiB).
-//   warps 2..9  dequant: raw int4 -> bf16 (subtract 8, then scale) into the A ring in
-//               the UMMA K-major 128-byte-swizzle layout, 16 rows per warp.
-//   warp 1      MMA: one thread issues tcgen05.mma (M = 128 weight rows, N = the
-//               block's routed rows rounded up to 16, K = 16 per instruction) into one
-//               of two TMEM accumulators of 256 columns, and tcgen05.commit frees the
-//               ring stages and publishes the accumulator.
-//   warps 10..17 epilogue (two per TMEM lane quadrant, alternate 16-column chunks):
-//               tcgen05.ld of the accumulator; SiLU(gate)*up written to the bf16
-//               intermediate (gate_up), or the expert output written to the per-slot
-//               fp32 buffer (down; the combine applies the top-k weight). Double
-//               buffering lets it overlap the next item.
+//   An item is (routing block b of up to 256 rows, a 256-row weight tile). CTA rank r of
+//   the pair owns the weight rows of 128-row tile 2*nt2 + r and, of the block's N routed
+//   rows (rounded up to 16), rows [r*N/2, (r+1)*N/2) of the activation operand. One
+//   M = 256 MMA then multiplies each CTA's 128 weight rows with all N rows, so each SM
+//   fetches only half of the activation bytes a single-CTA M = 128 tile would (those
+//   bytes, about 32 per MMA cycle per SM, come from L2 and their latency is what the
+//   rings must cover).
 //
-// The rings are sized at launch from the largest MMA N of the call: a B stage holds N
-// rows, and the shared memory a small N leaves free becomes a deeper A ring, so the
-// dequant warps can run further ahead of the MMA.
+//   warp 0      producer (both CTAs): per item one bulk copy of the packed codes +
+//               scales of two 128-wide K tiles of this CTA's weight tile into its raw
+//               ring, and per 64-wide K step its half of the block's activation rows as
+//               tiled TMA boxes (64, 16 and 8 rows, 128-byte swizzle) into its B ring;
+//               the copies of both CTAs complete on the B barrier of rank 0. The rows
+//               are contiguous because the activations are in routing order: the
+//               intermediate of the down projection already is, and the gate_up input is
+//               permuted into that order first.
+//   warps 2..9  dequant (both CTAs): raw int4 -> bf16 (subtract 8, then scale) into the
+//               A ring in the UMMA K-major 128-byte-swizzle layout, 16 rows per warp;
+//               arrivals go to rank 0's A barrier.
+//   warp 1      MMA (rank 0, one thread): tcgen05.mma.cta_group::2 (M = 256, N = the
+//               block's routed rows rounded up to 16, K = 16) into one of two TMEM
+//               accumulators of 256 columns; tcgen05.commit multicast to both CTAs frees
+//               the ring stages and publishes the accumulator.
+//   warps 10..17 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
+//               chunks): tcgen05.ld of this CTA's 128 accumulator rows; SiLU(gate)*up
+//               written to the bf16 intermediate (gate_up), or the expert output written
+//               to the per-slot fp32 buffer (down; the combine applies the top-k weight).
+//               Double buffering lets it overlap the next item.
+//
+// When the weight matrix has an odd number of 128-row tiles, rank 1 of the last pair
+// tile computes on stale shared memory and writes nothing.
 //
 // Operand orientation follows the blog's decode profile (dequantised weights in the
 // MMA-M slot, tokens in N): one dequantised weight tile serves every token of a block.
 // All waits are bounded; on timeout the CTA raises CHORD_DEV_TIMEOUT and unwinds after
-// waiting (bounded) for its copies and MMAs in flight, then frees TMEM.
+// waiting (bounded) for its copies and MMAs in flight, then frees TMEM. Both CTAs of a
+// pair meet at a cluster barrier before TMEM is freed and before either exits, so no
+// remote arrival or copy can target a CTA that has left.
 #include <cuda.h>
+
+#include <mutex>
 
 #include "tc_common.cuh"
 
@@ -54,9 +66,10 @@ constexpr int kTcThreads = 32 * (2 + kDequantWarps + kEpiWarps);
 
 constexpr int kAStageBytes = 128 * 64 * 2;
 constexpr int kRawStageBytes = kRawTiles * kTileBytes;
+constexpr int kBInFlightBytes = 96 * 1024;  // activation bytes to keep in flight per CTA
 
 struct TcDesc {
-  int e, nt, pos0, nvalid, end, pad[3];
+  int e, nt, pos0, nvalid, end, phantom, pad[2];
 };
 // fixed part (from the 1024-aligned base): descriptors, barriers, TMEM slot; then rings
 constexpr int kOffDesc = 0;
@@ -67,20 +80,21 @@ constexpr int kOffRings = 1024;
 static_assert(kOffTmemSlot + 16 <= kOffRings, "fixed part");
 constexpr int kSmemLimit = 232448 - 1024;  // 227 KiB opt-in per CTA, minus static shared
 
-// Ring geometry for a launch whose largest MMA N is nmax.
+// Ring geometry for a launch whose largest MMA N is nmax (each CTA holds nmax/2 rows of
+// a B stage).
 struct TcRings {
   int a_stages, b_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
 };
 __host__ __device__ inline TcRings tc_rings(int nmax) {
+  auto clamp = [](int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); };
   TcRings r;
-  r.b_stage_bytes = nmax * 128;
+  r.b_stage_bytes = (nmax / 2) * 128;
   const int avail = kSmemLimit - 1024 - kOffRings - kRawStages * kRawStageBytes;
-  // the activation ring covers TMA latency, so it gets every stage that fits next to a
-  // double-buffered A ring; what a small N leaves over deepens the A ring
-  int bs = (avail - 2 * kAStageBytes) / r.b_stage_bytes;
-  bs = bs < 2 ? 2 : (bs > kMaxStages ? kMaxStages : bs);
-  int as = (avail - bs * r.b_stage_bytes) / kAStageBytes;
-  as = as < 2 ? 2 : (as > kMaxStages ? kMaxStages : as);
+  // enough activation stages to cover the L2 latency, then as deep an A ring as fits
+  // (the dequant warps run ahead of the MMA), then whatever is left back to B
+  int bs = clamp((kBInFlightBytes + r.b_stage_bytes - 1) / r.b_stage_bytes, 2, kMaxStages);
+  const int as = clamp((avail - bs * r.b_stage_bytes) / kAStageBytes, 2, kMaxStages);
+  bs = clamp((avail - as * kAStageBytes) / r.b_stage_bytes, bs, kMaxStages);
   r.a_stages = as;
   r.b_stages = bs;
   r.off_a = kOffRings;
@@ -124,10 +138,10 @@ struct TcParams {
 };
 
 // Dequantises half hk (64 K) of one row's 128-K share into an A stage (UMMA K-major,
-// 128-byte swizzle). Lane (g, t) of dequant warp (rb, h) owns row r = rb*16 + 8h + g:
-// `c` holds its four code words (K slices j = 0..3 at offset 8t), `sp` the two scales
-// of slices 2hk, 2hk+1. The slice order alternates with g so the eight lanes of each
-// 16-byte store phase hit eight distinct bank groups.
+// 128-byte swizzle). Lane (g, t) owns row r: `c` holds its four code words (K slices
+// j = 0..3 at offset 8t), `sp` the two scales of slices 2hk, 2hk+1. The slice order
+// alternates with g so the eight lanes of each 16-byte store phase hit eight distinct
+// bank groups.
 template <int HK>
 __device__ __forceinline__ void dequant_row_half(const uint4& c, uint32_t sp, uint32_t a_stage, int r,
                                                  int g, int t) {
@@ -143,37 +157,29 @@ __device__ __forceinline__ void dequant_row_half(const uint4& c, uint32_t sp, ui
   }
 }
 
-// TMA: tiled box of the activation tensor (64 columns x box rows), 128-byte swizzle.
-__device__ __forceinline__ void tma_tile2d(uint32_t dst, const void* tmap, int col, int row, uint64_t* bar,
-                                           uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(row), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 template <int EPI>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap64, const __grid_constant__ CUtensorMap tmap16,
-                   TcParams p) {
+                   const __grid_constant__ CUtensorMap tmap8, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base for the swizzled operand stages
+  // 1024-byte aligned base for the swizzled operand stages (the same offset in both CTAs)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   const int AS = p.rings.a_stages, BS = p.rings.b_stages;
   const int b_stage_bytes = p.rings.b_stage_bytes;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + kRawStages;
-  uint64_t* a_full = raw_empty + kRawStages;
+  uint64_t* a_full = raw_empty + kRawStages;     // used in rank 0: both CTAs' dequant warps
   uint64_t* a_empty = a_full + kMaxStages;
-  uint64_t* b_full = a_empty + kMaxStages;
+  uint64_t* b_full = a_empty + kMaxStages;       // used in rank 0: both CTAs' copies
   uint64_t* b_empty = b_full + kMaxStages;
   uint64_t* acc_full = b_empty + kMaxStages;     // [2]
-  uint64_t* acc_empty = acc_full + 2;            // [2]
+  uint64_t* acc_empty = acc_full + 2;            // [2], used in rank 0: both epilogues
   uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
   uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
@@ -194,24 +200,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&raw_empty[s], kDequantWarps);
     }
     for (int s = 0; s < kMaxStages; ++s) {
-      mbar_init(&a_full[s], kDequantWarps);
+      mbar_init(&a_full[s], 2 * kDequantWarps);
       mbar_init(&a_empty[s], 1);
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     for (int d = 0; d < kDescRingTC; ++d) {
       mbar_init(&dfull[d], 1);
-      mbar_init(&dempty[d], kDequantWarps + 1 + kEpiWarps);
+      mbar_init(&dempty[d], kDequantWarps + kEpiWarps + (leader ? 1 : 0));
     }
     fence_barrier_init();
   }
   __syncthreads();
+  // both CTAs of a pair read the same header, so they leave here together or not at all
   if (abort_flag) return;
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  cluster_sync_all();  // the peer's barriers are initialised before anything arrives on them
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -220,6 +228,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int KT = p.K / kTileK;        // 128-wide raw steps
   const int NTILES = p.N / kTileN;
+  const int NT2 = (NTILES + 1) / 2;   // 256-row pair tiles
+  const int64_t cid = cluster_id_x(), ncl = num_clusters_x();
 
   if (warp == 0) {
     // ----------------------------------------------------------------- producer
@@ -227,9 +237,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ntp < 0) ntp = 0;
     if (ntp > p.cap) ntp = int(p.cap);
     const int64_t nblocks = ntp / p.block_m;
-    const int64_t items = nblocks * NTILES;
+    const int64_t items = nblocks * NT2;
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
+    const uint32_t b_full_l = cluster_addr(b_full, 0);
     uint32_t rstage = 0, nitem = 0;
     RingPos bpos;
     bool ok = true;
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int i = 0; i < kMaxN / 32; ++i) f[i] = -1;
       if (w >= items) return;
-      const int64_t b = w / NTILES;
+      const int64_t b = w / NT2;
       e = __ldg(p.expert_ids + b);
       const int pos0 = int(b * p.block_m);
 #pragma unroll
@@ -250,17 +261,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     };
     int e_next, f_next[kMaxN / 32];
-    load_meta(blockIdx.x, e_next, f_next);
-    for (int64_t w = blockIdx.x; ok; w += gridDim.x) {
+    load_meta(cid, e_next, f_next);
+    for (int64_t w = cid; ok; w += ncl) {
       const bool end = w >= items;
       int e = e_next, nt = 0, pos0 = 0, nvalid = 0;
       int fcur[kMaxN / 32];
 #pragma unroll
       for (int i = 0; i < kMaxN / 32; ++i) fcur[i] = f_next[i];
-      load_meta(w + gridDim.x, e_next, f_next);
+      load_meta(w + ncl, e_next, f_next);
       if (!end) {
-        nt = int(w % NTILES);
-        pos0 = int((w / NTILES) * p.block_m);
+        nt = int(w % NT2) * 2 + int(rank);
+        pos0 = int((w / NT2) * p.block_m);
         if (unsigned(e) < unsigned(p.E)) {
 #pragma unroll
           for (int i = 0; i < kMaxN / 32; ++i)
@@ -268,8 +279,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
-        if (nvalid == 0) continue;
+        if (nvalid == 0) continue;  // both CTAs see the same rows and skip together
       }
+      const bool phantom = nt >= NTILES;
       const uint32_t ds = nitem % kDescRingTC;
       if (nitem >= kDescRingTC &&
           !mbar_wait(&dempty[ds], ((nitem / kDescRingTC) - 1) & 1, abort_v, p.status))
@@ -280,12 +292,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         descs[ds].pos0 = pos0;
         descs[ds].nvalid = nvalid;
         descs[ds].end = end ? 1 : 0;
+        descs[ds].phantom = phantom ? 1 : 0;
         mbar_arrive(&dfull[ds]);
       }
       ++nitem;
       if (end) break;
       __syncwarp();
       const int nmma = (nvalid + 15) & ~15;
+      const int half = nmma >> 1;
+      const int row0 = pos0 + int(rank) * half;
       const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
       for (int kt0 = 0; kt0 < KT && ok; kt0 += kRawTiles) {
         const int ntl = min(kRawTiles, KT - kt0);
@@ -296,10 +311,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         if (lane == 0) {
-          uint8_t* st = smem + p.rings.off_raw + rs * kRawStageBytes;
-          mbar_arrive_expect_tx(&raw_full[rs], uint32_t(ntl) * kTileBytes);
-          bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &raw_full[rs],
-                        pol_w);
+          if (phantom) {
+            mbar_arrive(&raw_full[rs]);
+          } else {
+            uint8_t* st = smem + p.rings.off_raw + rs * kRawStageBytes;
+            mbar_arrive_expect_tx(&raw_full[rs], uint32_t(ntl) * kTileBytes);
+            bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &raw_full[rs],
+                          pol_w);
+          }
         }
         ++rstage;
         for (int sub = 0; sub < 2 * ntl; ++sub) {
@@ -310,12 +329,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
+            // rank 0 expects the bytes of both halves; each CTA copies its own half
+            if (leader) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
             const uint32_t bst = sbase + p.rings.off_b + s * b_stage_bytes;
+            const uint32_t bar = b_full_l + s * 8u;
             const int col = kt0 * kTileK + sub * 64;
             int r0 = 0;
-            for (; r0 + 64 <= nmma; r0 += 64) tma_tile2d(bst + r0 * 128, &tmap64, col, pos0 + r0, &b_full[s], pol_a);
-            for (; r0 < nmma; r0 += 16) tma_tile2d(bst + r0 * 128, &tmap16, col, pos0 + r0, &b_full[s], pol_a);
+            for (; r0 + 64 <= half; r0 += 64) tma_tile2d_pair(bst + r0 * 128, &tmap64, col, row0 + r0, bar, pol_a);
+            for (; r0 + 16 <= half; r0 += 16) tma_tile2d_pair(bst + r0 * 128, &tmap16, col, row0 + r0, bar, pol_a);
+            if (r0 < half) tma_tile2d_pair(bst + r0 * 128, &tmap8, col, row0 + r0, bar, pol_a);
           }
           bpos.next(BS);
         }
@@ -328,22 +350,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int dummy = 0;
       for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
         mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
-      // the last min(BS, fills) fills of the B ring, walking back from the current slot
-      RingPos back = bpos;
-      const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
-      for (uint32_t i = 0; i < n_back; ++i) {
-        if (back.slot == 0) {
-          back.slot = BS - 1;
-          back.phase ^= 1u;
-        } else {
-          --back.slot;
+      if (leader) {
+        // the last min(BS, fills) fills of the B ring (both halves complete on rank 0's
+        // barriers), walking back from the current slot
+        RingPos back = bpos;
+        const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
+        for (uint32_t i = 0; i < n_back; ++i) {
+          if (back.slot == 0) {
+            back.slot = BS - 1;
+            back.phase ^= 1u;
+          } else {
+            --back.slot;
+          }
+          mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
         }
-        mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (leader && lane == 0) {
       RingPos apos, bpos;
       uint64_t* last_bar = nullptr;
       uint32_t last_parity = 0;
@@ -357,12 +382,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, abort_v, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 256;
-        const uint32_t idesc = idesc_bf16_m128((d.nvalid + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_m256((d.nvalid + 15) & ~15);
         bool ok = true;
         for (int ks = 0; ks < 2 * KT; ++ks) {
           const uint32_t sa = apos.slot, pa = apos.phase;
           const uint32_t sb = bpos.slot, pb = bpos.phase;
-          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status) || !mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
+          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status) ||
+              !mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
             ok = false;
             break;
           }
@@ -371,17 +397,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t b_addr = sbase + p.rings.off_b + sb * b_stage_bytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
-                   (ks > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&a_empty[sa]);
-          tc_commit(&b_empty[sb]);
+            tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
+                    (ks > 0 || k > 0) ? 1u : 0u);
+          tc2_commit_both(&a_empty[sa]);
+          tc2_commit_both(&b_empty[sb]);
           last_bar = &b_empty[sb];
           last_parity = pb;
           apos.next(AS);
           bpos.next(BS);
         }
         if (!ok) break;
-        tc_commit(&acc_full[buf]);
+        tc2_commit_both(&acc_full[buf]);
       }
       // make sure no MMA is still writing TMEM before it is freed
       if (last_bar) {
@@ -393,6 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ----------------------------------------------------------------- dequant
     const int rb = warp - 2;
     const int g = lane >> 2, t = lane & 3;
+    const uint32_t a_full_l = cluster_addr(a_full, 0);
     uint32_t rstage = 0;
     RingPos apos;
     for (uint32_t it = 0;; ++it) {
@@ -433,7 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[s]);
+          if (lane == 0) mbar_arrive_cluster(a_full_l + s * 8u);
           apos.next(AS);
         }
         __syncwarp();
@@ -447,6 +474,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp & 3;                        // TMEM lane quadrant this warp may access
     const int half = (warp - 2 - kDequantWarps) >> 2;  // which 16-column chunks (even / odd)
     const int r = q * 32 + lane;
+    const uint32_t acc_empty_l = cluster_addr(acc_empty, 0);
     for (uint32_t it = 0;; ++it) {
       const uint32_t ds = it % kDescRingTC;
       if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
@@ -462,7 +490,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = 0; i < kMaxN / 32; ++i) {
         const int c = lane + 32 * i;
         f_col[i] = -1;
-        if (c < d.nvalid) {
+        if (c < d.nvalid && !d.phantom) {
           const int f = __ldg(p.sorted_ids + d.pos0 + c);
           if (f >= 0 && f < p.n_slots) f_col[i] = f;
         }
@@ -470,50 +498,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_v, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + buf * 256;
+      if (!d.phantom) {
 #pragma unroll
-      for (int cc = 0; cc < kMaxN / 16; ++cc) {
-        const int c0 = cc * 16;
-        if (c0 >= d.nvalid) break;
-        if ((cc & 1) != half) continue;
-        float v[16];
-        tmem_ld16(taddr + c0, v);
-        // column c0 + c lives in lane (c0 + c) % 32 of register set (c0 + c) / 32
-        const int src_set = c0 >> 5;
-        int f_set = f_col[0];
+        for (int cc = 0; cc < kMaxN / 16; ++cc) {
+          const int c0 = cc * 16;
+          if (c0 >= d.nvalid) break;
+          if ((cc & 1) != half) continue;
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          // column c0 + c lives in lane (c0 + c) % 32 of register set (c0 + c) / 32
+          const int src_set = c0 >> 5;
+          int f_set = f_col[0];
 #pragma unroll
-        for (int i = 1; i < kMaxN / 32; ++i)
-          if (src_set == i) f_set = f_col[i];
-        if (EPI == kGateUp) {
-          const bool gate = (r & 15) < 8;
-          const int i_col = d.nt * (kTileN / 2) + (r >> 4) * 8 + (r & 7);
+          for (int i = 1; i < kMaxN / 32; ++i)
+            if (src_set == i) f_set = f_col[i];
+          if (EPI == kGateUp) {
+            const bool gate = (r & 15) < 8;
+            const int i_col = d.nt * (kTileN / 2) + (r >> 4) * 8 + (r & 7);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
-            const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
-            if (gate && f >= 0)
-              p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
-          }
-        } else {
-          const int n = d.nt * kTileN + r;
+            for (int c = 0; c < 16; ++c) {
+              const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
+              const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
+              if (gate && f >= 0)
+                p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
+            }
+          } else {
+            const int n = d.nt * kTileN + r;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
-            if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c];
+            for (int c = 0; c < 16; ++c) {
+              const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
+              if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c];
+            }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive_cluster(acc_empty_l + buf * 8u);
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no MMA, copy or arrival of either CTA is still in flight
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -572,15 +604,61 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __res
   }
 }
 
+// Largest number of co-resident CTA pairs for this kernel and shared-memory size, per
+// device (clusters must fit inside a GPC, so this can be below half the SM count).
 template <int EPI>
-cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const TcParams& p, int grid,
-                       cudaStream_t stream) {
+int max_pairs(int smem_bytes, int max_ctas) {
+  struct Entry {
+    int dev, smem, pairs;
+  };
+  static std::mutex mu;
+  static Entry cache[16];
+  static int n_cache = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < n_cache; ++i)
+    if (cache[i].dev == dev && cache[i].smem == smem_bytes) return min(cache[i].pairs, max_ctas / 2);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(unsigned(max_ctas & ~1));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = size_t(smem_bytes);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int pairs = 0;
+  if (cudaOccupancyMaxActiveClusters(&pairs, tc_gemm_kernel<EPI>, &cfg) != cudaSuccess) return 0;
+  if (n_cache < 16) cache[n_cache++] = Entry{dev, smem_bytes, pairs};
+  return min(pairs, max_ctas / 2);
+}
+
+template <int EPI>
+cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const CUtensorMap& m8, const TcParams& p,
+                       int max_ctas, cudaStream_t stream) {
   auto kern = tc_gemm_kernel<EPI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kTcThreads, p.rings.smem_bytes, stream>>>(m64, m16, p);
+  const int pairs = max_pairs<EPI>(p.rings.smem_bytes, max_ctas);
+  if (pairs < 1) return cudaErrorLaunchOutOfResources;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(unsigned(2 * pairs));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = size_t(p.rings.smem_bytes);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, m64, m16, m8, p);
   count_launches(1);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace
@@ -615,27 +693,29 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
   }
-  CUtensorMap m64, m16;
+  CUtensorMap m64, m16, m8;
   cudaError_t err = make_tile_map(&m64, a.xs, a.cap, a.H, 64);
   if (err == cudaSuccess) err = make_tile_map(&m16, a.xs, a.cap, a.H, 16);
+  if (err == cudaSuccess) err = make_tile_map(&m8, a.xs, a.cap, a.H, 8);
   if (err != cudaSuccess) return err;
   p.blob = a.w13;
   p.tiles = a.w13 + blob_tiles_offset();
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
-  if ((err = launch_one<kGateUp>(m64, m16, p, grid, stream)) != cudaSuccess) return err;
+  if ((err = launch_one<kGateUp>(m64, m16, m8, p, grid, stream)) != cudaSuccess) return err;
   if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
 
   // down: W2 [E, H, I]; B rows of the intermediate a [cap, I], already in routing order
   if ((err = make_tile_map(&m64, a.a, a.cap, a.I, 64)) != cudaSuccess) return err;
   if ((err = make_tile_map(&m16, a.a, a.cap, a.I, 16)) != cudaSuccess) return err;
+  if ((err = make_tile_map(&m8, a.a, a.cap, a.I, 8)) != cudaSuccess) return err;
   p.blob = a.w2;
   p.tiles = a.w2 + blob_tiles_offset();
   p.N = a.H;
   p.K = a.I;
   p.role = CHORD_ROLE_DOWN;
-  return launch_one<kDown>(m64, m16, p, grid, stream);
+  return launch_one<kDown>(m64, m16, m8, p, grid, stream);
 }
 
 }  // namespace chord
