@@ -83,8 +83,10 @@ __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1
 // ------------------------------------------------------------------------------------
 // Workspace of chord_moe_forward:
 //   [status 256 B][a: cap x I bf16][y: T*topk x H fp32][xs: cap x H bf16]
-// a is the SiLU*up intermediate by sorted position, y the weighted expert outputs by
-// flat slot, xs the hidden rows in sorted order (tensor-core schedule only).
+// a is the SiLU*up intermediate by sorted position (row-major [cap, I] on the streaming
+// schedule, K-blocked [I/64][cap][64] on the tensor-core schedule), y the expert outputs
+// before the top-k weight by flat slot, xs the hidden rows in sorted order, K-blocked
+// [H/64][cap][64] (tensor-core schedule only).
 struct ForwardWorkspace {
   uint64_t a_offset, y_offset, xs_offset, total;
 };
@@ -304,9 +306,9 @@ struct ForwardArgs {
   const uint8_t* w13;
   const uint8_t* w2;
   uint16_t* out;
-  uint16_t* a;     // [cap, I] bf16 intermediate, indexed by sorted position
+  uint16_t* a;     // bf16 intermediate by sorted position: [cap, I], or [I/64][cap][64] (tensor core)
   float* y;        // [T*topk, H] fp32 expert outputs (before the top-k weight), by flat slot
-  uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
+  uint16_t* xs;    // [H/64][cap][64] bf16 hidden rows in sorted order (tensor-core schedule)
   uint32_t* status;
   int64_t T;
   int H, I, E, topk, block_m;

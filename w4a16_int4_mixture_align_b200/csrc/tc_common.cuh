@@ -113,15 +113,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// TMA into this CTA's shared memory: a tiled box (64 bf16 columns x the map's box rows,
-// 128-byte swizzle) of a 2-D tensor map; completion is signalled on the mbarrier at
-// cluster address `bar`, which may sit in either CTA of the pair. No multicast.
-__device__ __forceinline__ void tma_tile2d_pair(uint32_t dst, const void* tmap, int col, int row, uint32_t bar,
-                                                uint64_t policy) {
+// TMA into this CTA's shared memory: one box of a 3-D tensor map over a K-blocked
+// activation tensor [chunks][rows][64 bf16] (128-byte swizzle), starting at (column 0,
+// row, chunk); the box lands as [box chunks][box rows][128 B]. Completion is signalled on
+// the mbarrier at cluster address `bar`, which may sit in either CTA of the pair. No
+// multicast.
+__device__ __forceinline__ void tma_box3d_pair(uint32_t dst, const void* tmap, int row, int chunk, uint32_t bar,
+                                               uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(row), "r"(bar), "l"(policy)
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(0), "r"(row), "r"(chunk), "r"(bar), "l"(policy)
       : "memory");
 }
 

@@ -16,24 +16,27 @@
 //   bytes, about 32 per MMA cycle per SM, come from L2 and their latency is what the
 //   rings must cover).
 //
-//   warp 0      producer (both CTAs): per item one bulk copy of the packed codes +
-//               scales of two 128-wide K tiles of this CTA's weight tile into its raw
-//               ring, and per 64-wide K step its half of the block's activation rows as
-//               tiled TMA boxes (64, 16 and 8 rows, 128-byte swizzle) into its B ring;
-//               the copies of both CTAs complete on the B barrier of rank 0. The rows
-//               are contiguous because the activations are in routing order: the
-//               intermediate of the down projection already is, and the gate_up input is
-//               permuted into that order first.
-//   warps 2..9  dequant (both CTAs): raw int4 -> bf16 (subtract 8, then scale) into the
+//   warp 0      activation producer (both CTAs): per 128-wide K step one TMA request
+//               for this CTA's half of the block's rows, two 64-column chunks of them
+//               (a 3-D box of the K-blocked activation layout [K/64][rows][64], 128-byte
+//               swizzle), into its B ring; the copies of both CTAs complete on the B
+//               barrier of rank 0. One request per step matters: each TMA issue holds the
+//               issuing thread for a few hundred cycles, so the box height equals the
+//               half-block (a tensor map per height, 8..128 rows). The rows are contiguous
+//               because the activations are in routing order: the intermediate of the down
+//               projection is written that way, and the gate_up input is permuted first.
+//   warp 2      weight producer (both CTAs): one bulk copy of the packed codes + scales of
+//               two 128-wide K tiles of this CTA's weight tile per raw stage.
+//   warps 3..10 dequant (both CTAs): raw int4 -> bf16 (subtract 8, then scale) into the
 //               A ring in the UMMA K-major 128-byte-swizzle layout, 16 rows per warp;
 //               arrivals go to rank 0's A barrier.
 //   warp 1      MMA (rank 0, one thread): tcgen05.mma.cta_group::2 (M = 256, N = the
 //               block's routed rows rounded up to 16, K = 16) into one of two TMEM
 //               accumulators of 256 columns; tcgen05.commit multicast to both CTAs frees
 //               the ring stages and publishes the accumulator.
-//   warps 10..17 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
+//   warps 11..18 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
 //               chunks): tcgen05.ld of this CTA's 128 accumulator rows; SiLU(gate)*up
-//               written to the bf16 intermediate (gate_up), or the expert output written
+//               written to the K-blocked bf16 intermediate (gate_up), or the expert output written
 //               to the per-slot fp32 buffer (down; the combine applies the top-k weight).
 //               Double buffering lets it overlap the next item.
 //
@@ -62,7 +65,11 @@ constexpr int kMaxN = 256;
 constexpr int kDescRingTC = 8;
 constexpr int kDequantWarps = 8;
 constexpr int kEpiWarps = 8;
-constexpr int kTcThreads = 32 * (2 + kDequantWarps + kEpiWarps);
+constexpr int kTcThreads = 32 * (3 + kDequantWarps + kEpiWarps);
+constexpr int kFirstDequantWarp = 3;
+constexpr int kFirstEpiWarp = kFirstDequantWarp + kDequantWarps;
+constexpr int kBChunks = 2;        // 64-column chunks per activation request (one 128-K step)
+constexpr int kNumBoxMaps = 16;    // activation box heights 8, 16, ..., 128 rows
 
 constexpr int kAStageBytes = 128 * 64 * 2;
 constexpr int kRawStageBytes = kRawTiles * kTileBytes;
@@ -80,15 +87,15 @@ constexpr int kOffRings = 1024;
 static_assert(kOffTmemSlot + 16 <= kOffRings, "fixed part");
 constexpr int kSmemLimit = 232448 - 1024;  // 227 KiB opt-in per CTA, minus static shared
 
-// Ring geometry for a launch whose largest MMA N is nmax (each CTA holds nmax/2 rows of
-// a B stage).
+// Ring geometry for a launch whose largest MMA N is nmax (each CTA holds nmax/2 rows x
+// kBChunks chunks of a B stage).
 struct TcRings {
   int a_stages, b_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
 };
 __host__ __device__ inline TcRings tc_rings(int nmax) {
   auto clamp = [](int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); };
   TcRings r;
-  r.b_stage_bytes = (nmax / 2) * 128;
+  r.b_stage_bytes = (nmax / 2) * 128 * kBChunks;
   const int avail = kSmemLimit - 1024 - kOffRings - kRawStages * kRawStageBytes;
   // enough activation stages to cover the L2 latency, then as deep an A ring as fits
   // (the dequant warps run ahead of the MMA), then whatever is left back to B
@@ -157,10 +164,15 @@ __device__ __forceinline__ void dequant_row_half(const uint4& c, uint32_t sp, ui
   }
 }
 
+// Tensor maps of the K-blocked activation tensor [K/64][cap][64], one per box height
+// 8 * (i + 1) rows, box {64 columns, height, kBChunks chunks}.
+struct BoxMaps {
+  CUtensorMap m[kNumBoxMaps];
+};
+
 template <int EPI>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap64, const __grid_constant__ CUtensorMap tmap16,
-                   const __grid_constant__ CUtensorMap tmap8, TcParams p) {
+    tc_gemm_kernel(const __grid_constant__ BoxMaps maps, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled operand stages (the same offset in both CTAs)
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -199,6 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kDequantWarps);
     }
+    // descriptor consumers: dequant, epilogue, weight producer and (rank 0) the MMA thread
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&a_full[s], 2 * kDequantWarps);
       mbar_init(&a_empty[s], 1);
@@ -211,7 +224,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int d = 0; d < kDescRingTC; ++d) {
       mbar_init(&dfull[d], 1);
-      mbar_init(&dempty[d], kDequantWarps + kEpiWarps + (leader ? 1 : 0));
+      mbar_init(&dempty[d], kDequantWarps + kEpiWarps + 1 + (leader ? 1 : 0));
     }
     fence_barrier_init();
   }
@@ -232,16 +245,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int64_t cid = cluster_id_x(), ncl = num_clusters_x();
 
   if (warp == 0) {
-    // ----------------------------------------------------------------- producer
+    // ----------------------------------------------------------------- activation producer
     int ntp = *p.ntp;
     if (ntp < 0) ntp = 0;
     if (ntp > p.cap) ntp = int(p.cap);
     const int64_t nblocks = ntp / p.block_m;
     const int64_t items = nblocks * NT2;
-    const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
     const uint32_t b_full_l = cluster_addr(b_full, 0);
-    uint32_t rstage = 0, nitem = 0;
+    uint32_t nitem = 0;
     RingPos bpos;
     bool ok = true;
     // routing metadata of item w (its expert and the flat slots of this lane's 8 rows),
@@ -281,7 +293,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int o = 16; o > 0; o >>= 1) nvalid = max(nvalid, __shfl_xor_sync(0xffffffffu, nvalid, o));
         if (nvalid == 0) continue;  // both CTAs see the same rows and skip together
       }
-      const bool phantom = nt >= NTILES;
       const uint32_t ds = nitem % kDescRingTC;
       if (nitem >= kDescRingTC &&
           !mbar_wait(&dempty[ds], ((nitem / kDescRingTC) - 1) & 1, abort_v, p.status))
@@ -292,17 +303,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         descs[ds].pos0 = pos0;
         descs[ds].nvalid = nvalid;
         descs[ds].end = end ? 1 : 0;
-        descs[ds].phantom = phantom ? 1 : 0;
+        descs[ds].phantom = nt >= NTILES ? 1 : 0;
         mbar_arrive(&dfull[ds]);
       }
       ++nitem;
       if (end) break;
       __syncwarp();
       const int nmma = (nvalid + 15) & ~15;
-      const int half = nmma >> 1;
+      const int half = nmma >> 1;                 // rows per CTA, a multiple of 8
+      const CUtensorMap* map = &maps.m[(half >> 3) - 1];
       const int row0 = pos0 + int(rank) * half;
-      const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
-      for (int kt0 = 0; kt0 < KT && ok; kt0 += kRawTiles) {
+      for (int kb = 0; kb < KT; ++kb) {
+        const uint32_t s = bpos.slot;
+        // the slot's previous fill (one lap ago, opposite phase) must have been consumed
+        if (bpos.count >= uint32_t(BS) && !mbar_wait(&b_empty[s], bpos.phase ^ 1u, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          // rank 0 expects the bytes of both halves; each CTA copies its own half
+          if (leader) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u * kBChunks);
+          tma_box3d_pair(sbase + p.rings.off_b + s * b_stage_bytes, map, row0, kb * kBChunks, b_full_l + s * 8u,
+                         pol_a);
+        }
+        bpos.next(BS);
+      }
+      __syncwarp();
+    }
+    // drain: rank 0 waits (bounded, ignoring abort) for the last min(BS, fills) fills of
+    // the B ring (both halves complete on its barriers), walking back from the current slot
+    if (lane == 0 && leader) {
+      int dummy = 0;
+      RingPos back = bpos;
+      const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
+      for (uint32_t i = 0; i < n_back; ++i) {
+        if (back.slot == 0) {
+          back.slot = BS - 1;
+          back.phase ^= 1u;
+        } else {
+          --back.slot;
+        }
+        mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
+      }
+    }
+  } else if (warp == 2) {
+    // ----------------------------------------------------------------- weight producer
+    const uint64_t pol_w = policy_evict_first();
+    uint32_t rstage = 0;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t ds = it % kDescRingTC;
+      if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
+      const TcDesc d = descs[ds];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[ds]);
+      if (d.end) break;
+      const uint64_t tile0 = (uint64_t(d.e) * NTILES + d.nt) * KT;
+      bool ok = true;
+      for (int kt0 = 0; kt0 < KT; kt0 += kRawTiles) {
         const int ntl = min(kRawTiles, KT - kt0);
         const uint32_t rs = rstage % kRawStages;
         if (rstage >= uint32_t(kRawStages) &&
@@ -311,7 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         if (lane == 0) {
-          if (phantom) {
+          if (d.phantom) {
             mbar_arrive(&raw_full[rs]);
           } else {
             uint8_t* st = smem + p.rings.off_raw + rs * kRawStageBytes;
@@ -321,50 +378,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         ++rstage;
-        for (int sub = 0; sub < 2 * ntl; ++sub) {
-          const uint32_t s = bpos.slot;
-          // the slot's previous fill (one lap ago, opposite phase) must have been consumed
-          if (bpos.count >= uint32_t(BS) && !mbar_wait(&b_empty[s], bpos.phase ^ 1u, abort_v, p.status)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            // rank 0 expects the bytes of both halves; each CTA copies its own half
-            if (leader) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u);
-            const uint32_t bst = sbase + p.rings.off_b + s * b_stage_bytes;
-            const uint32_t bar = b_full_l + s * 8u;
-            const int col = kt0 * kTileK + sub * 64;
-            int r0 = 0;
-            for (; r0 + 64 <= half; r0 += 64) tma_tile2d_pair(bst + r0 * 128, &tmap64, col, row0 + r0, bar, pol_a);
-            for (; r0 + 16 <= half; r0 += 16) tma_tile2d_pair(bst + r0 * 128, &tmap16, col, row0 + r0, bar, pol_a);
-            if (r0 < half) tma_tile2d_pair(bst + r0 * 128, &tmap8, col, row0 + r0, bar, pol_a);
-          }
-          bpos.next(BS);
-        }
-        __syncwarp();
       }
       __syncwarp();
+      if (!ok) break;
     }
     // drain: wait (bounded, ignoring abort) for the copies still in flight
     if (lane == 0) {
       int dummy = 0;
       for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
         mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
-      if (leader) {
-        // the last min(BS, fills) fills of the B ring (both halves complete on rank 0's
-        // barriers), walking back from the current slot
-        RingPos back = bpos;
-        const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
-        for (uint32_t i = 0; i < n_back; ++i) {
-          if (back.slot == 0) {
-            back.slot = BS - 1;
-            back.phase ^= 1u;
-          } else {
-            --back.slot;
-          }
-          mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
-        }
-      }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
@@ -382,28 +404,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, abort_v, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 256;
-        const uint32_t idesc = idesc_bf16_m256((d.nvalid + 15) & ~15);
+        const int nmma = (d.nvalid + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_m256(nmma);
+        const uint32_t chunk_bytes = uint32_t(nmma >> 1) * 128u;  // one chunk of this CTA's rows
         bool ok = true;
-        for (int ks = 0; ks < 2 * KT; ++ks) {
-          const uint32_t sa = apos.slot, pa = apos.phase;
+        for (int kb = 0; kb < KT && ok; ++kb) {
           const uint32_t sb = bpos.slot, pb = bpos.phase;
-          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status) ||
-              !mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
+          if (!mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
           const uint32_t b_addr = sbase + p.rings.off_b + sb * b_stage_bytes;
+          for (int h = 0; h < kBChunks; ++h) {
+            const uint32_t sa = apos.slot, pa = apos.phase;
+            if (!mbar_wait(&a_full[sa], pa, abort_v, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
+            const uint32_t bh = b_addr + h * chunk_bytes;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
-                    (ks > 0 || k > 0) ? 1u : 0u);
-          tc2_commit_both(&a_empty[sa]);
+            for (int k = 0; k < 4; ++k)
+              tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(bh + k * 32), idesc,
+                      (kb > 0 || h > 0 || k > 0) ? 1u : 0u);
+            tc2_commit_both(&a_empty[sa]);
+            apos.next(AS);
+          }
+          if (!ok) break;
           tc2_commit_both(&b_empty[sb]);
           last_bar = &b_empty[sb];
           last_parity = pb;
-          apos.next(AS);
           bpos.next(BS);
         }
         if (!ok) break;
@@ -415,9 +446,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_wait(last_bar, last_parity, &dummy, p.status);
       }
     }
-  } else if (warp < 2 + kDequantWarps) {
+  } else if (warp < kFirstEpiWarp) {
     // ----------------------------------------------------------------- dequant
-    const int rb = warp - 2;
+    const int rb = warp - kFirstDequantWarp;
     const int g = lane >> 2, t = lane & 3;
     const uint32_t a_full_l = cluster_addr(a_full, 0);
     uint32_t rstage = 0;
@@ -472,7 +503,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ----------------------------------------------------------------- epilogue
     const int q = warp & 3;                        // TMEM lane quadrant this warp may access
-    const int half = (warp - 2 - kDequantWarps) >> 2;  // which 16-column chunks (even / odd)
+    const int half = (warp - kFirstEpiWarp) >> 2;  // which 16-column chunks (even / odd)
     const int r = q * 32 + lane;
     const uint32_t acc_empty_l = cluster_addr(acc_empty, 0);
     for (uint32_t it = 0;; ++it) {
@@ -520,7 +551,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
               const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
               if (gate && f >= 0)
-                p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
+                p.a_out[(int64_t(i_col >> 6) * p.cap + d.pos0 + c0 + c) * 64 + (i_col & 63)] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
             }
           } else {
@@ -568,22 +599,55 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (row-major), box 64 columns x box_rows rows, 128-byte
-// swizzle; rows past the end read as zero.
-cudaError_t make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int box_rows) {
+// Box maps of a K-blocked bf16 tensor [K/64][rows][64]: map i has box {64 columns,
+// 8 * (i + 1) rows, kBChunks chunks}, 128-byte swizzle; rows past the end read as zero.
+// Encoding sixteen maps costs host time, so the last few sets are kept, keyed by the
+// tensor's address and shape (the workspace of a layer is reused call after call).
+cudaError_t box_maps(BoxMaps* out, const void* base, int64_t rows, int K) {
+  struct Entry {
+    const void* base;
+    int64_t rows;
+    int K, dev;
+    BoxMaps maps;
+  };
+  static std::mutex mu;
+  static Entry cache[4];
+  static int n_cache = 0, next_slot = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < n_cache; ++i)
+    if (cache[i].base == base && cache[i].rows == rows && cache[i].K == K && cache[i].dev == dev) {
+      *out = cache[i].maps;
+      return cudaSuccess;
+    }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
-  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  BoxMaps maps;
+  cuuint64_t dims[3] = {64, cuuint64_t(rows), cuuint64_t(K / 64)};
+  cuuint64_t strides[2] = {128, cuuint64_t(rows) * 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  for (int i = 0; i < kNumBoxMaps; ++i) {
+    cuuint32_t box[3] = {64, cuuint32_t(8 * (i + 1)), cuuint32_t(kBChunks)};
+    CUresult r = fn(&maps.m[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  Entry& e = cache[next_slot];
+  e.base = base;
+  e.rows = rows;
+  e.K = K;
+  e.dev = dev;
+  e.maps = maps;
+  next_slot = (next_slot + 1) % 4;
+  if (n_cache < 4) ++n_cache;
+  *out = maps;
+  return cudaSuccess;
 }
 
-// xs[pos, :] = x[sorted_ids[pos] / topk, :] for every routed position (16 B per thread).
+// xs[c / 64][pos][c % 64] = x[sorted_ids[pos] / topk][c] for every routed position: the
+// hidden rows in routing order, K-blocked (16 B per thread).
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
                                                            const int32_t* __restrict__ sorted_ids,
                                                            const int32_t* __restrict__ ntp_p, int64_t cap,
@@ -600,7 +664,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __res
     const int f = __ldg(sorted_ids + pos);
     if (f < 0 || f >= n_slots) continue;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + int64_t(f / topk) * H + c));
-    *reinterpret_cast<uint4*>(xs + pos * H + c) = v;
+    *reinterpret_cast<uint4*>(xs + (int64_t(c >> 6) * cap + pos) * 64 + (c & 63)) = v;
   }
 }
 
@@ -637,8 +701,7 @@ int max_pairs(int smem_bytes, int max_ctas) {
 }
 
 template <int EPI>
-cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const CUtensorMap& m8, const TcParams& p,
-                       int max_ctas, cudaStream_t stream) {
+cudaError_t launch_one(const BoxMaps& maps, const TcParams& p, int max_ctas, cudaStream_t stream) {
   auto kern = tc_gemm_kernel<EPI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   if (err != cudaSuccess) return err;
@@ -656,7 +719,7 @@ cudaError_t launch_one(const CUtensorMap& m64, const CUtensorMap& m16, const CUt
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, m64, m16, m8, p);
+  err = cudaLaunchKernelEx(&cfg, kern, maps, p);
   count_launches(1);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
@@ -693,29 +756,25 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
   }
-  CUtensorMap m64, m16, m8;
-  cudaError_t err = make_tile_map(&m64, a.xs, a.cap, a.H, 64);
-  if (err == cudaSuccess) err = make_tile_map(&m16, a.xs, a.cap, a.H, 16);
-  if (err == cudaSuccess) err = make_tile_map(&m8, a.xs, a.cap, a.H, 8);
+  BoxMaps maps;
+  cudaError_t err = box_maps(&maps, a.xs, a.cap, a.H);
   if (err != cudaSuccess) return err;
   p.blob = a.w13;
   p.tiles = a.w13 + blob_tiles_offset();
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
-  if ((err = launch_one<kGateUp>(m64, m16, m8, p, grid, stream)) != cudaSuccess) return err;
+  if ((err = launch_one<kGateUp>(maps, p, grid, stream)) != cudaSuccess) return err;
   if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
 
-  // down: W2 [E, H, I]; B rows of the intermediate a [cap, I], already in routing order
-  if ((err = make_tile_map(&m64, a.a, a.cap, a.I, 64)) != cudaSuccess) return err;
-  if ((err = make_tile_map(&m16, a.a, a.cap, a.I, 16)) != cudaSuccess) return err;
-  if ((err = make_tile_map(&m8, a.a, a.cap, a.I, 8)) != cudaSuccess) return err;
+  // down: W2 [E, H, I]; B rows of the K-blocked intermediate a, already in routing order
+  if ((err = box_maps(&maps, a.a, a.cap, a.I)) != cudaSuccess) return err;
   p.blob = a.w2;
   p.tiles = a.w2 + blob_tiles_offset();
   p.N = a.H;
   p.K = a.I;
   p.role = CHORD_ROLE_DOWN;
-  return launch_one<kDown>(m64, m16, m8, p, grid, stream);
+  return launch_one<kDown>(maps, p, grid, stream);
 }
 
 }  // namespace chord
