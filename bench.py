@@ -299,7 +299,7 @@ def run_chord(args, rank, world, local_rank):
                    "routed_pairs": work["R"], "active_experts": work["active_experts"],
                    "l2": "no flush: weights %.2f GB > 126 MB L2" % (work["layer_bytes"] / 1e9),
                    "parallelism": f"replicas x{world}"},
-        "kernels_us": {"align": round(seg_ms[0] * 1000, 2), "gate_up": round(gu_us, 2),
+        "kernels_us": {"align+prep": round(seg_ms[0] * 1000, 2), "gate_up": round(gu_us, 2),
                        "down": round(dn_us, 2), "combine": round(seg_ms[3] * 1000, 2),
                        "gate_up+down": round(gu_us + dn_us, 2)},
         "layer": {"GB/s": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9, 1),

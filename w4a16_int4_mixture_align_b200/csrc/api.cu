@@ -303,12 +303,11 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
     if ((err = launch_validate(a, stream)) != cudaSuccess) return cuda_fail(err, "validate launch");
   }
   const bool timing = g_timing_on;
-  if (timing && (err = cudaEventRecord(g_timing[0], stream)) != cudaSuccess)
-    return cuda_fail(err, "timing event");
+  cudaEvent_t first = timing ? g_timing[0] : nullptr;
   const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) ||
                       (!(flags & CHORD_FLAG_FORCE_STREAM) && block_m > 32);
   cudaEvent_t mid = timing ? g_timing[1] : nullptr;
-  err = tensor ? launch_tc_gemms(a, stream, mid) : launch_stream_gemms(a, stream, mid);
+  err = tensor ? launch_tc_gemms(a, stream, first, mid) : launch_stream_gemms(a, stream, first, mid);
   if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");
   if (timing && (err = cudaEventRecord(g_timing[2], stream)) != cudaSuccess)
     return cuda_fail(err, "timing event");

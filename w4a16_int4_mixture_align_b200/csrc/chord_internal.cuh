@@ -321,8 +321,12 @@ void count_launches(int n);
 
 // `mid` (may be null) is recorded on the stream between the gate_up and down GEMMs.
 cudaError_t launch_validate(const ForwardArgs& a, cudaStream_t stream);
-cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid);
-cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid);
+// `first` (if set) is recorded right before the gate_up GEMM kernel, `mid` between the two
+// GEMM kernels.
+cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid);
+cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid);
+// xs <- the hidden rows in routing order, K-blocked [H/64][cap][64] (tensor-core schedule).
+cudaError_t launch_permute_rows(const ForwardArgs& a, cudaStream_t stream);
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream);
 
 }  // namespace chord

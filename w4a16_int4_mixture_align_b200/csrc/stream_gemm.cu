@@ -394,7 +394,7 @@ cudaError_t launch_tc(const StreamParams& p, int tc, int grid, cudaStream_t stre
 
 }  // namespace
 
-cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid) {
+cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid) {
   const int tc = a.block_m <= 8 ? 8 : (a.block_m <= 16 ? 16 : 32);
   const int grid = a.num_sms;
   StreamParams p{};
@@ -421,7 +421,9 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
   p.role = CHORD_ROLE_GATE_UP;
   p.act = a.x;
   p.act_ld = a.H;
-  cudaError_t err = launch_tc<kGateUp>(p, tc, grid, stream);
+  cudaError_t err = first ? cudaEventRecord(first, stream) : cudaSuccess;
+  if (err != cudaSuccess) return err;
+  err = launch_tc<kGateUp>(p, tc, grid, stream);
   if (err != cudaSuccess) return err;
   if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
 

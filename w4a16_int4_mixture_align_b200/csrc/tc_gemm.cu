@@ -646,28 +646,6 @@ cudaError_t box_maps(BoxMaps* out, const void* base, int64_t rows, int K) {
   return cudaSuccess;
 }
 
-// xs[c / 64][pos][c % 64] = x[sorted_ids[pos] / topk][c] for every routed position: the
-// hidden rows in routing order, K-blocked (16 B per thread).
-__global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
-                                                           const int32_t* __restrict__ sorted_ids,
-                                                           const int32_t* __restrict__ ntp_p, int64_t cap,
-                                                           int64_t n_slots, int topk, int H,
-                                                           uint16_t* __restrict__ xs) {
-  int64_t ntp = *ntp_p;
-  if (ntp < 0) ntp = 0;
-  if (ntp > cap) ntp = cap;
-  const int vec = H / 8;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < ntp * vec;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t pos = i / vec;
-    const int c = int(i % vec) * 8;
-    const int f = __ldg(sorted_ids + pos);
-    if (f < 0 || f >= n_slots) continue;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + int64_t(f / topk) * H + c));
-    *reinterpret_cast<uint4*>(xs + (int64_t(c >> 6) * cap + pos) * 64 + (c & 63)) = v;
-  }
-}
-
 // Largest number of co-resident CTA pairs for this kernel and shared-memory size, per
 // device (clusters must fit inside a GPC, so this can be below half the SM count).
 template <int EPI>
@@ -726,7 +704,7 @@ cudaError_t launch_one(const BoxMaps& maps, const TcParams& p, int max_ctas, cud
 
 }  // namespace
 
-cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t mid) {
+cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid) {
   TcParams p{};
   p.sorted_ids = a.sorted_ids;
   p.expert_ids = a.expert_ids;
@@ -746,24 +724,17 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
   const int grid = a.num_sms;
 
   // gate_up: W13 [E, 2I, H]; B rows from the hidden states permuted into routing order
-  {
-    const int64_t total = a.cap * (a.H / 8);
-    int64_t g = (total + 255) / 256;
-    if (g > int64_t(a.num_sms) * 16) g = int64_t(a.num_sms) * 16;
-    permute_rows_kernel<<<unsigned(g), 256, 0, stream>>>(a.x, a.sorted_ids, a.ntp, a.cap, a.T * a.topk, a.topk,
-                                                         a.H, a.xs);
-    count_launches(1);
-    cudaError_t e0 = cudaGetLastError();
-    if (e0 != cudaSuccess) return e0;
-  }
+  cudaError_t err = launch_permute_rows(a, stream);
+  if (err != cudaSuccess) return err;
   BoxMaps maps;
-  cudaError_t err = box_maps(&maps, a.xs, a.cap, a.H);
+  err = box_maps(&maps, a.xs, a.cap, a.H);
   if (err != cudaSuccess) return err;
   p.blob = a.w13;
   p.tiles = a.w13 + blob_tiles_offset();
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
+  if (first && (err = cudaEventRecord(first, stream)) != cudaSuccess) return err;
   if ((err = launch_one<kGateUp>(maps, p, grid, stream)) != cudaSuccess) return err;
   if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
 
