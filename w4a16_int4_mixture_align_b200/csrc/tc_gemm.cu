@@ -27,14 +27,16 @@
 //               projection is written that way, and the gate_up input is permuted first.
 //   warp 2      weight producer (both CTAs): one bulk copy of the packed codes + scales of
 //               two 128-wide K tiles of this CTA's weight tile per raw stage.
-//   warps 3..10 dequant (both CTAs): raw int4 -> bf16 (subtract 8, then scale) into the
-//               A ring in the UMMA K-major 128-byte-swizzle layout, 16 rows per warp;
-//               arrivals go to rank 0's A barrier.
+//   warps 3..18 dequant (both CTAs): raw int4 -> bf16 (subtract 8, then scale) into the
+//               A ring in the UMMA K-major 128-byte-swizzle layout, one row per lane, one
+//               128-wide K tile per A stage (the A and B rings step together); arrivals
+//               go to rank 0's A barrier. Sixteen warps, because the MMA waits on the
+//               latency of this dependent int -> bf16 chain rather than on issue slots.
 //   warp 1      MMA (rank 0, one thread): tcgen05.mma.cta_group::2 (M = 256, N = the
 //               block's routed rows rounded up to 16, K = 16) into one of two TMEM
 //               accumulators of 256 columns; tcgen05.commit multicast to both CTAs frees
 //               the ring stages and publishes the accumulator.
-//   warps 11..18 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
+//   warps 19..26 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
 //               chunks): tcgen05.ld of this CTA's 128 accumulator rows; SiLU(gate)*up
 //               written to the K-blocked bf16 intermediate (gate_up), or the expert output written
 //               to the per-slot fp32 buffer (down; the combine applies the top-k weight).
@@ -63,7 +65,7 @@ constexpr int kRawStages = 3;
 constexpr int kMaxStages = 8;     // upper bound of the A and B rings (runtime sized)
 constexpr int kMaxN = 256;
 constexpr int kDescRingTC = 8;
-constexpr int kDequantWarps = 8;
+constexpr int kDequantWarps = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = 32 * (3 + kDequantWarps + kEpiWarps);
 constexpr int kFirstDequantWarp = 3;
@@ -71,7 +73,8 @@ constexpr int kFirstEpiWarp = kFirstDequantWarp + kDequantWarps;
 constexpr int kBChunks = 2;        // 64-column chunks per activation request (one 128-K step)
 constexpr int kNumBoxMaps = 16;    // activation box heights 8, 16, ..., 128 rows
 
-constexpr int kAStageBytes = 128 * 64 * 2;
+constexpr int kAStageBytes = 128 * 128 * 2;   // 128 rows x one 128-K tile (two SW128 halves)
+constexpr int kAHalfBytes = kAStageBytes / 2;
 constexpr int kRawStageBytes = kRawTiles * kTileBytes;
 constexpr int kBInFlightBytes = 96 * 1024;  // activation bytes to keep in flight per CTA
 
@@ -88,7 +91,7 @@ static_assert(kOffTmemSlot + 16 <= kOffRings, "fixed part");
 constexpr int kSmemLimit = 232448 - 1024;  // 227 KiB opt-in per CTA, minus static shared
 
 // Ring geometry for a launch whose largest MMA N is nmax (each CTA holds nmax/2 rows x
-// kBChunks chunks of a B stage).
+// kBChunks chunks of a B stage). A and B stages both cover one 128-wide K step.
 struct TcRings {
   int a_stages, b_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
 };
@@ -144,11 +147,11 @@ struct TcParams {
   TcRings rings;
 };
 
-// Dequantises half hk (64 K) of one row's 128-K share into an A stage (UMMA K-major,
-// 128-byte swizzle). Lane (g, t) owns row r: `c` holds its four code words (K slices
-// j = 0..3 at offset 8t), `sp` the two scales of slices 2hk, 2hk+1. The slice order
-// alternates with g so the eight lanes of each 16-byte store phase hit eight distinct
-// bank groups.
+// Dequantises half hk (64 K) of one row's 128-K tile into one SW128 half of an A stage
+// (UMMA K-major, 128-byte swizzle). Lane (g, t) owns row r: `c` holds its four code
+// words (K slices j = 0..3 at offset 8t), `sp` the two scales of slices 2hk, 2hk+1. The
+// slice order alternates with g so the eight lanes of each 16-byte store phase hit eight
+// distinct bank groups.
 template <int HK>
 __device__ __forceinline__ void dequant_row_half(const uint4& c, uint32_t sp, uint32_t a_stage, int r,
                                                  int g, int t) {
@@ -414,24 +417,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
+          const uint32_t sa = apos.slot, pa = apos.phase;
+          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const uint32_t b_addr = sbase + p.rings.off_b + sb * b_stage_bytes;
+          const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
+#pragma unroll
           for (int h = 0; h < kBChunks; ++h) {
-            const uint32_t sa = apos.slot, pa = apos.phase;
-            if (!mbar_wait(&a_full[sa], pa, abort_v, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
-            const uint32_t bh = b_addr + h * chunk_bytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(bh + k * 32), idesc,
+              tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + h * kAHalfBytes + k * 32),
+                      sw128_kmajor_desc(b_addr + h * chunk_bytes + k * 32), idesc,
                       (kb > 0 || h > 0 || k > 0) ? 1u : 0u);
-            tc2_commit_both(&a_empty[sa]);
-            apos.next(AS);
           }
-          if (!ok) break;
+          tc2_commit_both(&a_empty[sa]);
+          apos.next(AS);
           tc2_commit_both(&b_empty[sb]);
           last_bar = &b_empty[sb];
           last_parity = pb;
@@ -448,8 +451,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < kFirstEpiWarp) {
     // ----------------------------------------------------------------- dequant
-    const int rb = warp - kFirstDequantWarp;
+    const int w = warp - kFirstDequantWarp;
+    const int rb = w >> 1, hrow = w & 1;          // 16-row block, upper or lower 8 rows
     const int g = lane >> 2, t = lane & 3;
+    const int row = rb * 16 + 8 * hrow + g;
     const uint32_t a_full_l = cluster_addr(a_full, 0);
     uint32_t rstage = 0;
     RingPos apos;
@@ -466,29 +471,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t rs = rstage % kRawStages;
         if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
         const uint32_t raw = sbase + p.rings.off_raw + rs * kRawStageBytes;
-        uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-        uint2 s0 = make_uint2(0, 0), s1 = s0;
-        for (int sub = 0; sub < 2 * ntl; ++sub) {
-          if ((sub & 1) == 0) {  // this lane's share of the next tile: rows rb*16+g and +8
-            const uint32_t tb = raw + (sub >> 1) * kTileBytes;
-            c0 = lds128(tb + rb * 1024 + g * 64 + t * 16);
-            c1 = lds128(tb + rb * 1024 + 512 + g * 64 + t * 16);
-            s0 = lds64(tb + kTileCodeBytes + rb * 128 + g * 16);
-            s1 = lds64(tb + kTileCodeBytes + rb * 128 + g * 16 + 8);
-          }
+        for (int tl = 0; tl < ntl; ++tl) {
+          // this lane's share of the tile: four code words and four group scales of its row
+          const uint32_t tb = raw + tl * kTileBytes;
+          const uint4 c = lds128(tb + rb * 1024 + hrow * 512 + g * 64 + t * 16);
+          const uint2 sc = lds64(tb + kTileCodeBytes + rb * 128 + g * 16 + hrow * 8);
           const uint32_t s = apos.slot;
           if (apos.count >= uint32_t(AS) && !mbar_wait(&a_empty[s], apos.phase ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
           }
           const uint32_t a_stage = sbase + p.rings.off_a + s * kAStageBytes;
-          if (sub & 1) {
-            dequant_row_half<1>(c0, s0.y, a_stage, rb * 16 + g, g, t);
-            dequant_row_half<1>(c1, s1.y, a_stage, rb * 16 + 8 + g, g, t);
-          } else {
-            dequant_row_half<0>(c0, s0.x, a_stage, rb * 16 + g, g, t);
-            dequant_row_half<0>(c1, s1.x, a_stage, rb * 16 + 8 + g, g, t);
-          }
+          dequant_row_half<0>(c, sc.x, a_stage, row, g, t);
+          dequant_row_half<1>(c, sc.y, a_stage + kAHalfBytes, row, g, t);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(a_full_l + s * 8u);
