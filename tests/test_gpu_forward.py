@@ -141,6 +141,15 @@ def test_no_local_slot_gives_zero_rows(chord, path):
     assert np.all(bf16_bits_to_f64(got) == 0)
 
 
+@pytest.mark.parametrize("path", ["stream", "tensor"])
+def test_topk_above_one_warp(chord, path):
+    # top-k 40 of 64 experts: the combine holds slots 32..39 in a second lane set
+    d = small_inputs(9, E=64, topk=40, H=256, I=128)
+    flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR
+    got = run_layer(make_layer(chord, d, block_m=16), d, flags)
+    assert_layer_close(got, oracle_rows(d, None))
+
+
 def test_single_expert_topk1(chord):
     d = small_inputs(33, E=1, topk=1)
     got = run_layer(make_layer(chord, d, block_m=8), d)

@@ -11,7 +11,7 @@
 // popcount of its lower peers, and the lowest peer advances the expert's running
 // position. Runs are ordered by a prefix over per-run histograms.
 //
-//   n <= 32 x 1024 : one CTA of 32 warps (runs of ceil(n/1024) steps) does count, scan,
+//   n <= 4 x 1024  : one CTA of 32 warps (runs of ceil(n/1024) steps) does count, scan,
 //                    scatter and fill (1 launch)
 //   larger n       : count kernel (per-chunk histograms) -> scan kernel (1 CTA) ->
 //                    scatter + fill kernel, histograms in the caller's workspace.
@@ -23,6 +23,10 @@ namespace {
 constexpr int kChunk = 1024;       // flat slots per warp chunk
 constexpr int kSteps = kChunk / 32;
 constexpr int kMaxE = 1024;
+// Up to this many 1024-slot chunks the routing sort runs in one CTA (one launch); above
+// it the count / scan / scatter kernels spread the slots over the GPU (one CTA sorting
+// 32 chunks took ~70 us).
+constexpr int kSingleMaxChunks = 4;
 
 __device__ __forceinline__ bool is_local(int e, int E) { return unsigned(e) < unsigned(E); }
 
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
 
 size_t align_workspace_bytes(int64_t n, int E) {
   const int64_t G = (n + kChunk - 1) / kChunk;
-  if (G <= 32) return 0;
+  if (G <= kSingleMaxChunks) return 0;
   return align256(uint64_t(E) * G * 4) + align256(uint64_t(E) * 4) + align256(uint64_t(E + 1) * 4);
 }
 
@@ -282,7 +286,7 @@ cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int6
                          int64_t nblocks, int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntp,
                          int32_t* offsets, void* workspace, cudaStream_t stream) {
   const int64_t G = (n + kChunk - 1) / kChunk;
-  if (G <= 32) {
+  if (G <= kSingleMaxChunks) {
     const size_t smem = (size_t(32) * E + E + E + 1 + 33) * sizeof(int);
     cudaError_t err = cudaFuncSetAttribute(align_single_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

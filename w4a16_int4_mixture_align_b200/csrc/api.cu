@@ -288,6 +288,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   a.a = reinterpret_cast<uint16_t*>(wsb + ws.a_offset);
   a.y = reinterpret_cast<float*>(wsb + ws.y_offset);
   a.xs = reinterpret_cast<uint16_t*>(wsb + ws.xs_offset);
+  a.slot_pos = reinterpret_cast<int32_t*>(wsb + ws.slot_pos_offset);
   a.status = reinterpret_cast<uint32_t*>(wsb);
   a.T = T;
   a.H = H;
@@ -306,6 +307,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   cudaEvent_t first = timing ? g_timing[0] : nullptr;
   const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) ||
                       (!(flags & CHORD_FLAG_FORCE_STREAM) && block_m > 32);
+  a.y_blocked = tensor;
   cudaEvent_t mid = timing ? g_timing[1] : nullptr;
   err = tensor ? launch_tc_gemms(a, stream, first, mid) : launch_stream_gemms(a, stream, first, mid);
   if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");

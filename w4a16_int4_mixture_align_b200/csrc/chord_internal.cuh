@@ -82,13 +82,16 @@ __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1
 
 // ------------------------------------------------------------------------------------
 // Workspace of chord_moe_forward:
-//   [status 256 B][a: cap x I bf16][y: T*topk x H fp32][xs: cap x H bf16]
+//   [status 256 B][a: cap x I bf16][y: cap x H fp32][xs: cap x H bf16][slot_pos: T*topk i32]
 // a is the SiLU*up intermediate by sorted position (row-major [cap, I] on the streaming
-// schedule, K-blocked [I/64][cap][64] on the tensor-core schedule), y the expert outputs
-// before the top-k weight by flat slot, xs the hidden rows in sorted order, K-blocked
-// [H/64][cap][64] (tensor-core schedule only).
+// schedule, K-blocked [I/64][cap][64] on the tensor-core schedule); y the expert outputs
+// before the top-k weight (by flat slot [T*topk, H] on the streaming schedule, by sorted
+// position in 128-column blocks [H/128][cap][128] on the tensor-core schedule, so that a
+// work item writes one contiguous block); xs the hidden rows in sorted order, K-blocked
+// [H/64][cap][64], and slot_pos the sorted position of every local flat slot (both
+// tensor-core schedule only).
 struct ForwardWorkspace {
-  uint64_t a_offset, y_offset, xs_offset, total;
+  uint64_t a_offset, y_offset, xs_offset, slot_pos_offset, total;
 };
 __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int topk, int E, int H,
                                                               int I, int block_m) {
@@ -96,8 +99,9 @@ __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int top
   int64_t cap = T * topk + int64_t(E) * (block_m - 1);
   w.a_offset = 256;
   w.y_offset = align256(w.a_offset + uint64_t(cap) * I * 2);
-  w.xs_offset = align256(w.y_offset + uint64_t(T) * topk * H * 4);
-  w.total = align256(w.xs_offset + uint64_t(cap) * H * 2);
+  w.xs_offset = align256(w.y_offset + uint64_t(cap) * H * 4);
+  w.slot_pos_offset = align256(w.xs_offset + uint64_t(cap) * H * 2);
+  w.total = align256(w.slot_pos_offset + uint64_t(T) * topk * 4);
   return w;
 }
 
@@ -307,8 +311,11 @@ struct ForwardArgs {
   const uint8_t* w2;
   uint16_t* out;
   uint16_t* a;     // bf16 intermediate by sorted position: [cap, I], or [I/64][cap][64] (tensor core)
-  float* y;        // [T*topk, H] fp32 expert outputs (before the top-k weight), by flat slot
+  float* y;        // fp32 expert outputs before the top-k weight: [T*topk, H] by flat slot, or
+                   // [H/128][cap][128] by sorted position (y_blocked, tensor core)
   uint16_t* xs;    // [H/64][cap][64] bf16 hidden rows in sorted order (tensor-core schedule)
+  int32_t* slot_pos;  // [T*topk] sorted position of each local flat slot (tensor-core schedule)
+  bool y_blocked;     // y is by sorted position in 128-column blocks
   uint32_t* status;
   int64_t T;
   int H, I, E, topk, block_m;

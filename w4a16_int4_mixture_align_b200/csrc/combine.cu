@@ -1,9 +1,10 @@
 // combine.cu -- top-k weighted combine and optional routing validation.
 //
-// The down kernels write y[f, :] = W2[e] . a for every local flat slot f. The combine
-// multiplies each row by its top-k weight and sums over the token's local slots in
-// ascending slot order in FP32 (acc += w_j * y_j), then rounds once to BF16; a token with
-// no local slot gets a zero row.
+// The down kernels write the expert output W2[e] . a of every local flat slot f (by slot
+// on the streaming schedule, by sorted position on the tensor-core schedule). The combine
+// multiplies each by its top-k weight and sums over the token's local slots in ascending
+// slot order in FP32 (acc += w_j * y_j), then rounds once to BF16; a token with no local
+// slot gets a zero row.
 // The blog excludes this step from its kernel timings ("Messungen"); here it is one
 // HBM-bound pass reading T*topk_local*H*4 bytes and writing T*H*2 bytes.
 #include "chord_internal.cuh"
@@ -11,41 +12,86 @@
 namespace chord {
 namespace {
 
-// One thread per 8 consecutive outputs of one token.
-__global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ topk_ids,
-                                                      const float* __restrict__ topk_weights,
-                                                      const float* __restrict__ y,
-                                                      uint16_t* __restrict__ out, int64_t T,
-                                                      int H, int topk, int E) {
-  const int vec_per_row = H / 8;
-  const int64_t total = T * vec_per_row;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t t = i / vec_per_row;
-    const int c = int(i % vec_per_row) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < topk; ++j) {
-      const int e = __ldg(topk_ids + t * topk + j);
-      if (unsigned(e) >= unsigned(E)) continue;
-      const float w = __ldg(topk_weights + t * topk + j);
-      const float4* src = reinterpret_cast<const float4*>(y + (t * topk + j) * int64_t(H) + c);
-      const float4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
-      // product rounded, then added (no fused multiply-add), as the layer is defined
-      acc[0] = __fadd_rn(acc[0], __fmul_rn(w, v0.x)); acc[1] = __fadd_rn(acc[1], __fmul_rn(w, v0.y));
-      acc[2] = __fadd_rn(acc[2], __fmul_rn(w, v0.z)); acc[3] = __fadd_rn(acc[3], __fmul_rn(w, v0.w));
-      acc[4] = __fadd_rn(acc[4], __fmul_rn(w, v1.x)); acc[5] = __fadd_rn(acc[5], __fmul_rn(w, v1.y));
-      acc[6] = __fadd_rn(acc[6], __fmul_rn(w, v1.z)); acc[7] = __fadd_rn(acc[7], __fmul_rn(w, v1.w));
+constexpr int kCombineThreads = 128;
+constexpr int kCombineVecs = 2;                    // 8-output vectors per thread and item
+constexpr int kCombineCols = kCombineThreads * 8 * kCombineVecs;  // outputs per work item
+
+// Work item = (token t, 2048 consecutive outputs); a thread owns two vectors of 8 outputs,
+// 1024 apart, so each slot's loads come in independent pairs. Lane j % 32
+// of every warp holds slot j's weight and row of y (top-k up to 64), and each output
+// accumulates its token's local slots in ascending j. BLOCKED selects y by sorted position
+// in 128-column blocks [H/128][cap][128] (tensor-core schedule) instead of y by flat slot
+// [T*topk, H] (streaming schedule).
+template <bool BLOCKED>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const int32_t* __restrict__ topk_ids, const float* __restrict__ topk_weights,
+    const float* __restrict__ y, const int32_t* __restrict__ slot_pos, uint16_t* __restrict__ out, int64_t T,
+    int H, int topk, int E, int64_t cap) {
+  const int lane = threadIdx.x & 31;
+  const int nchunk = (H + kCombineCols - 1) / kCombineCols;
+  for (int64_t item = blockIdx.x; item < T * nchunk; item += gridDim.x) {
+    const int64_t t = item / nchunk;
+    const int c0 = int(item % nchunk) * kCombineCols + threadIdx.x * 8;
+    // slot j's row of y (lane j % 32 of set j / 32), or -1 when the slot is not local (or
+    // its position is unknown)
+    int64_t row[2] = {-1, -1};
+    float w[2] = {0.f, 0.f};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = h * 32 + lane;
+      if (j < topk) {
+        const int64_t f = t * topk + j;
+        const int e = __ldg(topk_ids + f);
+        if (unsigned(e) < unsigned(E)) {
+          w[h] = __ldg(topk_weights + f);
+          if (BLOCKED) {
+            const int pos = __ldg(slot_pos + f);
+            row[h] = (pos >= 0 && pos < cap) ? pos : -1;
+          } else {
+            row[h] = f;
+          }
+        }
+      }
     }
-    uint4 o;
-    o.x = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[0]))) |
-          (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[1]))) << 16);
-    o.y = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[2]))) |
-          (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[3]))) << 16);
-    o.z = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[4]))) |
-          (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[5]))) << 16);
-    o.w = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[6]))) |
-          (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[7]))) << 16);
-    *reinterpret_cast<uint4*>(out + t * H + c) = o;
+    float acc[kCombineVecs][8];
+#pragma unroll
+    for (int u = 0; u < kCombineVecs; ++u)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+    for (int j = 0; j < topk; ++j) {
+      const int64_t rj = __shfl_sync(0xffffffffu, j < 32 ? row[0] : row[1], j & 31);
+      const float wj = __shfl_sync(0xffffffffu, j < 32 ? w[0] : w[1], j & 31);
+      if (rj < 0) continue;
+      float4 v[kCombineVecs][2];
+#pragma unroll
+      for (int u = 0; u < kCombineVecs; ++u) {
+        const int c = c0 + u * kCombineThreads * 8;
+        v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < H) {
+          const float* src = BLOCKED ? y + ((int64_t(c >> 7) * cap + rj) << 7) + (c & 127) : y + rj * H + c;
+          v[u][0] = __ldcs(reinterpret_cast<const float4*>(src));
+          v[u][1] = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+        }
+      }
+      // product rounded, then added (no fused multiply-add), as the layer is defined
+#pragma unroll
+      for (int u = 0; u < kCombineVecs; ++u) {
+        const float vv[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(wj, vv[i]));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineVecs; ++u) {
+      const int c = c0 + u * kCombineThreads * 8;
+      if (c >= H) continue;
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[u][2 * i]))) |
+               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[u][2 * i + 1]))) << 16);
+      *reinterpret_cast<uint4*>(out + t * H + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -78,12 +124,15 @@ __global__ void validate_kernel(const int32_t* __restrict__ topk_ids,
 }  // namespace
 
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
-  const int64_t total = a.T * (a.H / 8);
-  if (total == 0) return cudaSuccess;
-  int64_t grid = (total + 255) / 256;
+  if (a.T == 0) return cudaSuccess;
+  int64_t grid = a.T * ((a.H + kCombineCols - 1) / kCombineCols);
   if (grid > int64_t(a.num_sms) * 16) grid = int64_t(a.num_sms) * 16;
-  combine_kernel<<<unsigned(grid), 256, 0, stream>>>(a.topk_ids, a.topk_weights, a.y, a.out, a.T, a.H,
-                                                      a.topk, a.E);
+  if (a.y_blocked)
+    combine_kernel<true><<<unsigned(grid), kCombineThreads, 0, stream>>>(
+        a.topk_ids, a.topk_weights, a.y, a.slot_pos, a.out, a.T, a.H, a.topk, a.E, a.cap);
+  else
+    combine_kernel<false><<<unsigned(grid), kCombineThreads, 0, stream>>>(
+        a.topk_ids, a.topk_weights, a.y, a.slot_pos, a.out, a.T, a.H, a.topk, a.E, a.cap);
   count_launches(1);
   return cudaGetLastError();
 }

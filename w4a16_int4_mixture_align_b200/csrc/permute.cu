@@ -5,9 +5,14 @@
 // sorted_ids (the routing sort of the Chord blog's indexed path), K-blocked as
 // [H/64][cap][64]: xs[c / 64][pos][c % 64] = x[sorted_ids[pos] / topk][c]. Padding
 // positions (sentinel slots) are skipped; the GEMMs never read them back into a result.
+// The same pass records slot_pos[f] = pos, the inverse of sorted_ids over the local
+// slots, with which the combine finds a slot's expert output in the position-ordered y.
 //
 // One warp copies one routed row: 32 lanes read 512 contiguous bytes of the source row
-// per step and write them as four 128-byte runs, one per 64-column chunk.
+// per step and write them as four 128-byte runs, one per 64-column chunk. A hidden row is
+// read once per local slot of its token (up to top-k times), so the reads ask L2 to keep
+// it (evict_last) while the copies, larger than L2, stream out (evict_first). (Staging 32
+// rows in shared memory to write 4 KiB runs measured slower: fewer CTAs and two phases.)
 #include "chord_internal.cuh"
 
 namespace chord {
@@ -15,9 +20,22 @@ namespace {
 
 constexpr int kPermuteWarps = 8;
 
+__device__ __forceinline__ uint4 ldg_keep(const void* p, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void stg_stream(void* p, const uint4& v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w), "l"(pol)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(32 * kPermuteWarps) permute_rows_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ ntp_p,
-    int64_t cap, int64_t n_slots, int topk, int H, uint16_t* __restrict__ xs) {
+    int64_t cap, int64_t n_slots, int topk, int H, uint16_t* __restrict__ xs, int32_t* __restrict__ slot_pos) {
   int64_t ntp = *ntp_p;
   if (ntp < 0) ntp = 0;
   if (ntp > cap) ntp = cap;
@@ -25,15 +43,17 @@ __global__ void __launch_bounds__(32 * kPermuteWarps) permute_rows_kernel(
   const int64_t warp0 = int64_t(blockIdx.x) * kPermuteWarps + (threadIdx.x >> 5);
   const int64_t nwarps = int64_t(gridDim.x) * kPermuteWarps;
   const int vec = H / 8;  // 16-byte vectors per row
+  const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
   for (int64_t pos = warp0; pos < ntp; pos += nwarps) {
     const int f = __ldg(sorted_ids + pos);
     if (f < 0 || f >= n_slots) continue;
+    if (lane == 0) slot_pos[f] = int32_t(pos);
     const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(f / topk) * H);
     uint16_t* dst = xs + pos * 64;
     for (int v = lane; v < vec; v += 32) {
-      const uint4 val = __ldg(src + v);
+      const uint4 val = ldg_keep(src + v, keep);
       const int c = v * 8;
-      *reinterpret_cast<uint4*>(dst + int64_t(c >> 6) * cap * 64 + (c & 63)) = val;
+      stg_stream(dst + int64_t(c >> 6) * cap * 64 + (c & 63), val, stream);
     }
   }
 }
@@ -45,7 +65,8 @@ cudaError_t launch_permute_rows(const ForwardArgs& a, cudaStream_t stream) {
   if (ctas > int64_t(a.num_sms) * 8) ctas = int64_t(a.num_sms) * 8;
   if (ctas < 1) ctas = 1;
   permute_rows_kernel<<<unsigned(ctas), 32 * kPermuteWarps, 0, stream>>>(a.x, a.sorted_ids, a.ntp, a.cap,
-                                                                         a.T * a.topk, a.topk, a.H, a.xs);
+                                                                         a.T * a.topk, a.topk, a.H, a.xs,
+                                                                         a.slot_pos);
   count_launches(1);
   return cudaGetLastError();
 }

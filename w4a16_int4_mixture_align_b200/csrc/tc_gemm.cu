@@ -38,8 +38,9 @@
 //               the ring stages and publishes the accumulator.
 //   warps 19..26 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
 //               chunks): tcgen05.ld of this CTA's 128 accumulator rows; SiLU(gate)*up
-//               written to the K-blocked bf16 intermediate (gate_up), or the expert output written
-//               to the per-slot fp32 buffer (down; the combine applies the top-k weight).
+//               written to the K-blocked bf16 intermediate (gate_up), or the fp32 expert
+//               output written by sorted position in 128-column blocks (down; the combine
+//               applies the top-k weight).
 //               Double buffering lets it overlap the next item.
 //
 // When the weight matrix has an odd number of 128-row tiles, rank 1 of the last pair
@@ -550,11 +551,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
             }
           } else {
-            const int n = d.nt * kTileN + r;
+            // y by sorted position in 128-column blocks: this item's tile is one
+            // contiguous run of 512-byte rows
+            float* yb = p.y_out + (int64_t(d.nt) * p.cap + d.pos0 + c0) * kTileN + r;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
-              if (f >= 0) p.y_out[int64_t(f) * p.H + n] = v[c];
+              if (f >= 0) yb[c * kTileN] = v[c];
             }
           }
         }
