@@ -98,6 +98,15 @@ __device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb
     c1[u] = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
     sv[u] = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + g * 16);
   }
+  // the tile's activation fragments, issued together ahead of the dequantisation so their
+  // L1 latency overlaps it
+  uint4 xv[NTILE][4][NT8];
+#pragma unroll
+  for (int u = 0; u < NTILE; ++u)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8) xv[u][j][n8] = ldg_nc128(xrow[n8] + (t0 + 2 * u) * kTileK + 32 * j + 8 * t);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -114,9 +123,8 @@ __device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb
       const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
 #pragma unroll
       for (int n8 = 0; n8 < NT8; ++n8) {
-        const uint4 xv = ldg_nc128(xrow[n8] + (t0 + 2 * u) * kTileK + 32 * j + 8 * t);
-        mma_bf16_16816(acc[n8][(2 * u) % NSET], a_lo, xv.x, xv.y);
-        mma_bf16_16816(acc[n8][(2 * u + 1) % NSET], a_hi, xv.z, xv.w);
+        mma_bf16_16816(acc[n8][(2 * u) % NSET], a_lo, xv[u][j][n8].x, xv[u][j][n8].y);
+        mma_bf16_16816(acc[n8][(2 * u + 1) % NSET], a_hi, xv[u][j][n8].z, xv[u][j][n8].w);
       }
     }
   }
