@@ -49,6 +49,8 @@ def _load():
         lib.oracle_align_blocks.argtypes = [i64, i64, i64, i64]
         lib.oracle_align_blocks.restype = i64
         lib.oracle_moe_align.argtypes = [i32p, i64, i64, i64, i64, i32p, i32p, i32p, i32p]
+        lib.oracle_router_topk.restype = ctypes.c_int
+        lib.oracle_router_topk.argtypes = [f32p, i64, i64, i64, i32p, f32p]
         lib.oracle_moe_align.restype = ctypes.c_int
         lib.oracle_moe_forward.argtypes = [u16p, i32p, f32p, i32p, u16p, i32p, u16p,
                                            i64, i64, i64, i64, i64, ctypes.c_void_p, i64,
@@ -106,6 +108,21 @@ def moe_align(topk_ids: np.ndarray, E: int, block_m: int):
     if rc != 0:
         raise ValueError(f"oracle_moe_align failed ({rc})")
     return sorted_ids, expert_ids, int(ntp[0]), offs
+
+
+def router_topk(logits: np.ndarray, topk: int):
+    """Router upstream of the routing sort: (topk_ids int32 [T, k] global expert ids,
+    topk_weights float32 [T, k]), the top-k logits (ties to the lower id) and their
+    softmax renormalised over the chosen ones."""
+    lib = _load()
+    lg = np.ascontiguousarray(logits, dtype=np.float32)
+    T, G = lg.shape
+    ids = np.empty((T, topk), dtype=np.int32)
+    w = np.empty((T, topk), dtype=np.float32)
+    rc = lib.oracle_router_topk(_ptr(lg), T, G, topk, _ptr(ids), _ptr(w))
+    if rc != 0:
+        raise ValueError(f"oracle_router_topk failed ({rc})")
+    return ids, w
 
 
 def moe_forward(x, topk_ids, topk_weights, qw13, s13, qw2, s2, rows=None, n_threads=0):

@@ -23,6 +23,11 @@
  *   act      a = bf16_rne( silu(h[i]) * h[I+i] ), gate rows first, up rows second.
  *   down     y = a . W2[e]^T, FP32 accumulation.
  *   combine  out[t] = bf16_rne( sum over local slots j, ascending, of w[t,j] * y_j ).
+ *   router   (the step upstream of align, for the fused routing entry point) per token
+ *            the topk largest logits, ties to the lower expert id, and their softmax
+ *            renormalised over the chosen ones: w_r = exp(l_r - l_0) / sum_j exp(l_j - l_0)
+ *            (the layer's problem statement: top-k softmax routing, weights renormalised;
+ *            the full softmax denominator cancels in the renormalisation).
  *
  * Every floating-point reduction runs in plain ascending order in FP32; this file is
  * built with -ffp-contract=off so no multiply-add is fused.
@@ -229,5 +234,43 @@ int oracle_moe_forward(const uint16_t* x, const int32_t* topk_ids, const float* 
     }
   }
   free(w13); free(w2); free(y); free(pairs); free(h); free(a); free(xf);
+  return 0;
+}
+
+/* Router (see the header): topk_ids[t, r] = expert of rank r (descending logit, ties to
+ * the lower id), topk_weights[t, r] = exp(l_r - l_0) / sum_j exp(l_j - l_0), in double,
+ * summed in rank order, rounded once to float. Returns 0, or -1 for bad arguments. */
+int oracle_router_topk(const float* logits, int64_t T, int64_t G, int64_t k, int32_t* topk_ids,
+                       float* topk_weights) {
+  if (T < 0 || G < 1 || k < 1 || k > G) return -1;
+  unsigned char* taken = (unsigned char*)malloc((size_t)G);
+  double* e = (double*)malloc((size_t)k * sizeof(double));
+  if (!taken || !e) {
+    free(taken);
+    free(e);
+    return -1;
+  }
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * G;
+    memset(taken, 0, (size_t)G);
+    for (int64_t r = 0; r < k; ++r) {
+      int64_t best = -1;
+      for (int64_t g = 0; g < G; ++g) {
+        if (taken[g]) continue;
+        if (best < 0 || l[g] > l[best]) best = g; /* strictly greater: ties keep the lower id */
+      }
+      taken[best] = 1;
+      topk_ids[t * k + r] = (int32_t)best;
+    }
+    const double l0 = (double)l[topk_ids[t * k]];
+    double sum = 0.0;
+    for (int64_t r = 0; r < k; ++r) {
+      e[r] = exp((double)l[topk_ids[t * k + r]] - l0);
+      sum += e[r];
+    }
+    for (int64_t r = 0; r < k; ++r) topk_weights[t * k + r] = (float)(e[r] / sum);
+  }
+  free(taken);
+  free(e);
   return 0;
 }

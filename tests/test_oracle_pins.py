@@ -386,3 +386,47 @@ def test_oracle_reproduces_golden_fixture():
     assert s.tolist() == g["sorted_ids"] and eids.tolist() == g["expert_ids"]
     assert offs.tolist() == g["expert_offsets"]
     assert np.array_equal(run_oracle(d), g["out"])
+
+
+# ------------------------------------------------------------------------------ router
+
+def _router_brute(logits, k):
+    """Library routines only: a stable argsort of the negated logits (ties keep the lower
+    expert id) and scipy's softmax over the chosen logits."""
+    from scipy.special import softmax
+    order = np.argsort(-logits.astype(np.float64), axis=1, kind="stable")[:, :k]
+    chosen = np.take_along_axis(logits.astype(np.float64), order, axis=1)
+    return order.astype(np.int32), softmax(chosen, axis=1)
+
+
+@pytest.mark.parametrize("G,k", [(384, 8), (100, 3), (64, 64), (7, 1)])
+def test_router_matches_sort_and_softmax(G, k):
+    rng = np.random.default_rng(11 + G + k)
+    logits = rng.standard_normal((257, G)).astype(np.float32)
+    # coarse values in some rows create ties, which must go to the lower id
+    logits[::5] = np.round(logits[::5] * 2) / 2
+    ids, w = oracle.router_topk(logits, k)
+    ref_ids, ref_w = _router_brute(logits, k)
+    np.testing.assert_array_equal(ids, ref_ids)
+    np.testing.assert_allclose(w, ref_w, rtol=2e-7, atol=0)
+
+
+def test_router_closed_forms():
+    # all logits equal: the k lowest ids, weight exactly 1/k each
+    ids, w = oracle.router_topk(np.full((3, 40), 0.25, np.float32), 5)
+    assert np.all(ids == np.arange(5)) and np.all(w == np.float32(1 / 5))
+    # k = number of experts: the full softmax, experts by descending logit
+    lg = np.array([[0.0, 1.0, -2.0, 3.0]], np.float32)
+    ids, w = oracle.router_topk(lg, 4)
+    e = np.exp(lg[0].astype(np.float64))
+    np.testing.assert_array_equal(ids[0], [3, 1, 0, 2])
+    np.testing.assert_allclose(w[0], (e / e.sum())[[3, 1, 0, 2]], rtol=2e-7)
+    # adding a constant to every logit (exactly, here) changes nothing
+    rng = np.random.default_rng(5)
+    base = (rng.integers(-64, 64, (50, 96)) / 8).astype(np.float32)
+    i0, w0 = oracle.router_topk(base, 8)
+    i1, w1 = oracle.router_topk(base + np.float32(4.0), 8)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_allclose(w0, w1, rtol=2e-7)
+    # weights of a row sum to one
+    np.testing.assert_allclose(w0.astype(np.float64).sum(axis=1), 1.0, rtol=1e-6)
