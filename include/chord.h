@@ -107,6 +107,34 @@ CHORD_API chord_status_t chord_moe_align(const int32_t* topk_ids /* device [T, t
                                int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
                                size_t workspace_bytes, chord_stream_t stream);
 
+/* ----------------------------------------------------------------------------------
+ * chord_router_topk_align: the router step upstream of moe_align, fused with it.
+ *
+ * The layer's problem statement routes by top-k softmax with the weights renormalised
+ * over the chosen experts; the Chord blog leaves routing outside its kernel timings
+ * ("Messungen") and feeds the indexed path vLLM's sorted routing ("Zwei
+ * Kernel-Familien"). Per token t:
+ *   topk_ids[t, r]     = the expert with the r-th largest logit (r = 0 .. topk-1), ties to
+ *                        the lower expert id; GLOBAL ids in [0, E_global);
+ *   topk_weights[t, r] = exp(l_r - l_0) / sum_j exp(l_j - l_0), i.e. the softmax over all
+ *                        logits renormalised over the chosen ones (fp32);
+ * then exactly the routing tensors of chord_moe_align(topk_ids, T, topk, E, block_m, ...)
+ * for the local experts [0, E) (ids >= E belong to other shards).
+ *
+ * logits: device fp32 [T, E_global], finite or -inf. topk_ids / topk_weights: device
+ * [T, topk] int32 / fp32 outputs. The other arguments, limits and the workspace rule are
+ * those of chord_moe_align, plus topk <= E_global <= 1024. Up to 8 tokens run as ONE
+ * launch (the CTA that routes the tokens also sorts them); larger batches run a routing
+ * kernel (one warp per token) and the sort kernels. Returns CHORD_ERR_UNSUPPORTED for
+ * E_global out of range.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API chord_status_t chord_router_topk_align(const float* logits, int64_t T, int E_global, int topk, int E,
+                                                 int block_m, int32_t* topk_ids, float* topk_weights,
+                                                 int32_t* sorted_ids, int32_t* expert_ids,
+                                                 int32_t* num_tokens_padded /* [1] */,
+                                                 int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
+                                                 size_t workspace_bytes, chord_stream_t stream);
+
 /* Routing sort for callers that cannot allocate device memory (no counterpart on the
  * pages). Same arguments, results and limits as chord_moe_align, minus the workspace:
  * the scratch that large batches need lives in a static device array of 576 KiB that

@@ -54,6 +54,7 @@ SIGNATURES = {
                                _SZ, _I, _P]),
     "chord_moe_check_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "chord_moe_align_noalloc": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "chord_router_topk_align": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
 }
@@ -158,6 +159,18 @@ def chord_moe_align_noalloc(topk_ids, E, block_m, sorted_ids, expert_ids, num_to
                                          _ptr(expert_ids), _ptr(num_tokens_padded),
                                          _ptr(expert_offsets), _stream(stream)),
            "chord_moe_align_noalloc")
+
+
+def chord_router_topk_align(logits, topk, E, block_m, topk_ids, topk_weights, sorted_ids, expert_ids,
+                            num_tokens_padded, expert_offsets=None, workspace=None, stream=None):
+    """Top-k softmax router (fp32 logits [T, E_global] -> global topk_ids, renormalised
+    topk_weights) fused with the routing sort over the local experts [0, E)."""
+    T, E_global = logits.shape
+    ws_bytes = 0 if workspace is None else _nbytes(workspace)
+    _check(lib().chord_router_topk_align(_ptr(logits), T, E_global, topk, E, block_m, _ptr(topk_ids),
+                                         _ptr(topk_weights), _ptr(sorted_ids), _ptr(expert_ids),
+                                         _ptr(num_tokens_padded), _ptr(expert_offsets), _ptr(workspace),
+                                         ws_bytes, _stream(stream)), "chord_router_topk_align")
 
 
 def chord_repack_weights(qweight, scales, role, out, group_size=32, stream=None):

@@ -15,6 +15,8 @@
 //                    scatter and fill (1 launch)
 //   larger n       : count kernel (per-chunk histograms) -> scan kernel (1 CTA) ->
 //                    scatter + fill kernel, histograms in the caller's workspace.
+#include <math.h>
+
 #include "chord_internal.cuh"
 
 namespace chord {
@@ -157,12 +159,12 @@ __device__ void fill_tail(const int* cnt, const int* off, int E, int block_m, in
   }
 }
 
-// ---- single CTA (n <= 32 chunks) ---------------------------------------------------
-__global__ void __launch_bounds__(1024) align_single_kernel(
+// ---- single CTA (n <= kSingleMaxChunks chunks) ---------------------------------------
+// The whole sort by one CTA of 1024 threads; `smem` holds (32 + 2) * E + 34 ints.
+__device__ __forceinline__ void align_single_body(
     const int32_t* __restrict__ ids, int64_t n, int E, int block_m, int64_t cap, int64_t nblocks,
     int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntp_out,
-    int32_t* __restrict__ offsets_out) {
-  extern __shared__ int smem[];
+    int32_t* __restrict__ offsets_out, int* smem) {
   int* hist = smem;                 // [32][E]
   int* cnt = hist + 32 * E;         // [E]
   int* off = cnt + E;               // [E+1]
@@ -202,6 +204,138 @@ __global__ void __launch_bounds__(1024) align_single_kernel(
   if (offsets_out)
     for (int e = tid; e <= E; e += blockDim.x) offsets_out[e] = off[e];
 }
+
+__global__ void __launch_bounds__(1024) align_single_kernel(
+    const int32_t* __restrict__ ids, int64_t n, int E, int block_m, int64_t cap, int64_t nblocks,
+    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntp_out,
+    int32_t* __restrict__ offsets_out) {
+  extern __shared__ int smem[];
+  align_single_body(ids, n, E, block_m, cap, nblocks, sorted_ids, expert_ids, ntp_out, offsets_out, smem);
+}
+
+// ---- router: top-k softmax routing, one warp per token ------------------------------
+// Lane l holds the logits of experts l, l + 32, ... (PER slots). Each lane keeps its
+// best unselected slot; every round the warp takes the largest of them (larger value,
+// or the lower id on equal values), and only the lane that supplied it rescans. Lane
+// r % 32 ends with the expert of rank r (descending logit, ties to the lower id).
+constexpr int kRouterMaxG = 1024;
+constexpr int kNoExpert = 0x7fffffff;
+
+template <int PER>
+__device__ __forceinline__ void router_token(const float* __restrict__ row, int G, int k, int lane,
+                                             int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
+  float v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < G ? __ldg(row + e) : -INFINITY;
+  }
+  uint32_t taken = 0;
+  // this lane's best unselected slot (ascending e: strictly greater keeps the lower id)
+  auto local_best = [&](float& bv, int& bi) {
+    bv = -INFINITY;
+    bi = kNoExpert;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      if (e < G && !((taken >> i) & 1u) && (bi == kNoExpert || v[i] > bv)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+  };
+  float lv;
+  int li;
+  local_best(lv, li);
+  int id_a = 0, id_b = 0;  // ranks lane and 32 + lane
+  float l_a = -INFINITY, l_b = -INFINITY;
+  for (int r = 0; r < k; ++r) {
+    float bv = lv;
+    int bi = li;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != kNoExpert && (bi == kNoExpert || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (r == lane) {
+      id_a = bi;
+      l_a = bv;
+    } else if (r == lane + 32) {
+      id_b = bi;
+      l_b = bv;
+    }
+    if (li == bi) {  // this lane supplied the winner: mark it and find its next best
+      taken |= 1u << (bi >> 5);
+      local_best(lv, li);
+    }
+  }
+  // weights: softmax over the chosen logits, relative to the largest (rank 0)
+  const float l0 = __shfl_sync(0xffffffffu, l_a, 0);
+  const float e_a = lane < k ? expf(l_a - l0) : 0.f;
+  const float e_b = lane + 32 < k ? expf(l_b - l0) : 0.f;
+  float part = e_a + e_b;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if (lane < k) {
+    ids_out[lane] = id_a;
+    w_out[lane] = e_a / part;
+  }
+  if (lane + 32 < k) {
+    ids_out[lane + 32] = id_b;
+    w_out[lane + 32] = e_b / part;
+  }
+}
+
+template <int PER>
+__device__ __forceinline__ void route_tokens(const float* __restrict__ logits, int64_t T, int G, int k,
+                                             int32_t* __restrict__ topk_ids, float* __restrict__ topk_weights,
+                                             int64_t warp0, int64_t nwarps, int lane) {
+  for (int64_t t = warp0; t < T; t += nwarps)
+    router_token<PER>(logits + t * G, G, k, lane, topk_ids + t * k, topk_weights + t * k);
+}
+
+// Slots per lane: the smallest instantiated count that covers G.
+__device__ __forceinline__ void route_tokens_any(const float* __restrict__ logits, int64_t T, int G, int k,
+                                                 int32_t* __restrict__ topk_ids, float* __restrict__ topk_weights,
+                                                 int64_t warp0, int64_t nwarps, int lane) {
+  const int per = (G + 31) / 32;
+  if (per <= 4) route_tokens<4>(logits, T, G, k, topk_ids, topk_weights, warp0, nwarps, lane);
+  else if (per <= 8) route_tokens<8>(logits, T, G, k, topk_ids, topk_weights, warp0, nwarps, lane);
+  else if (per <= 12) route_tokens<12>(logits, T, G, k, topk_ids, topk_weights, warp0, nwarps, lane);
+  else if (per <= 16) route_tokens<16>(logits, T, G, k, topk_ids, topk_weights, warp0, nwarps, lane);
+  else route_tokens<32>(logits, T, G, k, topk_ids, topk_weights, warp0, nwarps, lane);
+}
+
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int64_t T, int G,
+                                                          int k, int32_t* __restrict__ topk_ids,
+                                                          float* __restrict__ topk_weights) {
+  route_tokens_any(logits, T, G, k, topk_ids, topk_weights,
+                   int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5),
+                   int64_t(gridDim.x) * (blockDim.x >> 5), threadIdx.x & 31);
+}
+
+// Router and sort fused in one CTA, for batches of at most 8 tokens: the warps route the
+// tokens, then the CTA sorts the ids it has just written (visible after the barrier).
+// Larger batches route on many CTAs first: measured, one SM routing 32 tokens took 4 us
+// more than a routing kernel plus the sort, while up to 8 tokens the saved launch wins.
+constexpr int kFusedMaxTokens = 8;
+
+__global__ void __launch_bounds__(1024) router_align_single_kernel(
+    const float* __restrict__ logits, int64_t T, int G, int k, int32_t* __restrict__ topk_ids,
+    float* __restrict__ topk_weights, int E, int block_m, int64_t cap, int64_t nblocks,
+    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntp_out,
+    int32_t* __restrict__ offsets_out) {
+  extern __shared__ int smem[];
+  route_tokens_any(logits, T, G, k, topk_ids, topk_weights, threadIdx.x >> 5, blockDim.x >> 5, threadIdx.x & 31);
+  __syncthreads();
+  align_single_body(topk_ids, T * k, E, block_m, cap, nblocks, sorted_ids, expert_ids, ntp_out, offsets_out,
+                    smem);
+}
+
 
 // ---- multi CTA ---------------------------------------------------------------------
 // workspace: chunk_hist [E][G] int32 | cnt [E] | off [E+1]
@@ -314,6 +448,33 @@ cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int6
       ids, n, E, block_m, G, cap, nblocks, chunk_hist, cnt, off, sorted_ids, expert_ids);
   count_launches(3);
   return cudaGetLastError();
+}
+
+cudaError_t launch_router_align(const float* logits, int64_t T, int G, int k, int32_t* topk_ids,
+                                float* topk_weights, int E, int block_m, int64_t cap, int64_t nblocks,
+                                int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntp, int32_t* offsets,
+                                void* workspace, cudaStream_t stream) {
+  const int64_t n = T * k;
+  const int64_t G_chunks = (n + kChunk - 1) / kChunk;
+  if (T <= kFusedMaxTokens && G_chunks <= kSingleMaxChunks) {
+    const size_t smem = (size_t(32) * E + E + E + 1 + 33) * sizeof(int);
+    cudaError_t err = cudaFuncSetAttribute(router_align_single_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err != cudaSuccess) return err;
+    router_align_single_kernel<<<1, 1024, smem, stream>>>(logits, T, G, k, topk_ids, topk_weights, E, block_m, cap,
+                                                          nblocks, sorted_ids, expert_ids, ntp, offsets);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+  int64_t ctas = (T + 7) / 8;
+  const int64_t max_ctas = 148 * 8;
+  if (ctas > max_ctas) ctas = max_ctas;
+  router_topk_kernel<<<unsigned(ctas), 256, 0, stream>>>(logits, T, G, k, topk_ids, topk_weights);
+  count_launches(1);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_align(topk_ids, n, E, block_m, cap, nblocks, sorted_ids, expert_ids, ntp, offsets, workspace,
+                      stream);
 }
 
 }  // namespace chord

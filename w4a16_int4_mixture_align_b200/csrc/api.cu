@@ -146,6 +146,33 @@ chord_status_t chord_moe_align(const int32_t* topk_ids, int64_t T, int topk, int
   return CHORD_OK;
 }
 
+chord_status_t chord_router_topk_align(const float* logits, int64_t T, int E_global, int topk, int E,
+                                       int block_m, int32_t* topk_ids, float* topk_weights, int32_t* sorted_ids,
+                                       int32_t* expert_ids, int32_t* num_tokens_padded, int32_t* expert_offsets,
+                                       void* workspace, size_t workspace_bytes, chord_stream_t stream) {
+  g_detail[0] = 0;
+  chord_status_t st = check_align_args(T, topk, E, block_m);
+  if (st != CHORD_OK) return st;
+  if (E_global < topk || E_global > 1024)
+    return fail(CHORD_ERR_UNSUPPORTED, "E_global=%d outside [topk=%d, 1024]", E_global, topk);
+  if ((T > 0 && (!logits || !topk_ids || !topk_weights)) || !sorted_ids || !expert_ids || !num_tokens_padded)
+    return fail(CHORD_ERR_INVALID_ARG, "null routing pointer");
+  const size_t need = align_workspace_bytes(T * topk, E);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "align workspace needs %zu bytes, got %zu", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (need > 0 && !aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  const int64_t cap = chord_moe_align_capacity(T, topk, E, block_m);
+  const int64_t nblocks = chord_moe_align_num_blocks(T, topk, E, block_m);
+  cudaError_t err = launch_router_align(logits, T, E_global, topk, topk_ids, topk_weights, E, block_m, cap,
+                                        nblocks, sorted_ids, expert_ids, num_tokens_padded, expert_offsets,
+                                        workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "router + moe_align launch");
+  return CHORD_OK;
+}
+
 size_t chord_repacked_bytes(int E, int N, int K, int group_size) {
   if (E < 1 || N < 1 || K < 1 || group_size != kGroup || N % kTileN || K % kTileK) return 0;
   return size_t(blob_total_bytes(E, N, K));

@@ -293,6 +293,11 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int64_t cap,
                          int64_t nblocks, int32_t* sorted_ids, int32_t* expert_ids,
                          int32_t* ntp, int32_t* offsets, void* workspace, cudaStream_t stream);
+// Top-k softmax router then the routing sort (one launch when T*k is small).
+cudaError_t launch_router_align(const float* logits, int64_t T, int G, int k, int32_t* topk_ids,
+                                float* topk_weights, int E, int block_m, int64_t cap, int64_t nblocks,
+                                int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntp, int32_t* offsets,
+                                void* workspace, cudaStream_t stream);
 size_t align_workspace_bytes(int64_t n, int E);
 
 cudaError_t launch_repack(const int32_t* qweight, const uint16_t* scales, int E, int N, int K,
