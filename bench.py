@@ -260,6 +260,10 @@ def run_chord(args, rank, world, local_rank):
     barrier(world)
     sampler.stop()
     e2e_ms = s2.elapsed_time(e2)
+
+    # ---- the fused router + routing sort at this workload's shape (outside the timed
+    # regions above; graph-replayed, so host marshalling does not hide device time)
+    router_us = time_router(chord, cfg, rcfg, dev)
     h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
     d2h = out_h.numel() * 2
 
@@ -310,8 +314,48 @@ def run_chord(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": sampler.summary(t_wall0, t_wall1),
+        "router_topk_align": {"us_per_call": round(router_us, 2),
+                              "what": "chord_router_topk_align on fp32 logits [T, E_global], top-%d, "
+                                      "then the routing sort (not part of value)" % cfg.topk},
     }
     return line
+
+
+def time_router(chord, cfg, rcfg, dev, calls=20, replays=10):
+    """Device µs per chord_router_topk_align call on seeded N(0,1) logits of the workload's
+    shape, from CUDA-graph replays of `calls` back-to-back calls."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(rcfg.seed)
+    T, G, k, E = cfg.T, cfg.E_global, cfg.topk, cfg.E
+    bm = chord.chord_select_block_m(T, k, E, G, cfg.H, cfg.I)
+    logits = torch.randn((T, G), dtype=torch.float32, device=dev, generator=g)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    s = torch.empty(chord.chord_moe_align_capacity(T, k, E, bm), dtype=torch.int32, device=dev)
+    e = torch.empty(max(chord.chord_moe_align_num_blocks(T, k, E, bm), 1), dtype=torch.int32, device=dev)
+    n = torch.empty(1, dtype=torch.int32, device=dev)
+    wsb = chord.chord_moe_align_workspace_bytes(T, k, E)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev) if wsb else None
+    side = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            chord.chord_router_topk_align(logits, k, E, bm, ids, w, s, e, n, None, ws)
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(calls):
+                chord.chord_router_topk_align(logits, k, E, bm, ids, w, s, e, n, None, ws)
+        graph.replay()
+        side.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(side)
+        for _ in range(replays):
+            graph.replay()
+        b.record(side)
+        side.synchronize()
+    del graph
+    return a.elapsed_time(b) * 1000.0 / (calls * replays)
 
 
 def max_over_ranks(vals, world, device=None):
