@@ -43,6 +43,15 @@
 //               applies the top-k weight).
 //               Double buffering lets it overlap the next item.
 //
+// The A and B rings step together (one 128-K step per stage), so they share one barrier
+// ring indexed by step (depth D = the deeper of the two): step_full[j % D] collects the
+// 32 dequant-warp arrivals of both CTAs and the activation bytes of step j, and one
+// multicast commit per step frees step_empty[j % D] for both rings. Neither producer can
+// fill step j + D before step j is done (D is at least either ring's depth), so a phase
+// never receives arrivals from two steps. One wait and one commit per step keep the MMA
+// thread's own work short: its MMA issue blocks for about the tensor time, so whatever
+// else it does between steps is a bubble in the tensor pipe.
+//
 // When the weight matrix has an odd number of 128-row tiles, rank 1 of the last pair
 // tile computes on stale shared memory and writes nothing.
 //
@@ -183,6 +192,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   const int AS = p.rings.a_stages, BS = p.rings.b_stages;
+  const int DS = AS > BS ? AS : BS;  // depth of the step barrier ring
   const int b_stage_bytes = p.rings.b_stage_bytes;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
@@ -190,11 +200,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + kRawStages;
-  uint64_t* a_full = raw_empty + kRawStages;     // used in rank 0: both CTAs' dequant warps
-  uint64_t* a_empty = a_full + kMaxStages;
-  uint64_t* b_full = a_empty + kMaxStages;       // used in rank 0: both CTAs' copies
-  uint64_t* b_empty = b_full + kMaxStages;
-  uint64_t* acc_full = b_empty + kMaxStages;     // [2]
+  uint64_t* step_full = raw_empty + kRawStages;  // [D] used in rank 0: dequant arrivals + copies
+  uint64_t* step_empty = step_full + kMaxStages; // [D] one multicast commit per step
+  uint64_t* spare = step_empty + kMaxStages;     // [2 * kMaxStages] unused
+  uint64_t* acc_full = spare + 2 * kMaxStages;   // [2]
   uint64_t* acc_empty = acc_full + 2;            // [2], used in rank 0: both epilogues
   uint64_t* dfull = acc_empty + 2;               // [kDescRingTC]
   uint64_t* dempty = dfull + kDescRingTC;        // [kDescRingTC]
@@ -217,10 +226,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // descriptor consumers: dequant, epilogue, weight producer and (rank 0) the MMA thread
     for (int s = 0; s < kMaxStages; ++s) {
-      mbar_init(&a_full[s], 2 * kDequantWarps);
-      mbar_init(&a_empty[s], 1);
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+      mbar_init(&step_full[s], 2 * kDequantWarps + 1);  // dequant warps of both CTAs + rank 0's copy
+      mbar_init(&step_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -256,9 +263,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t nblocks = ntp / p.block_m;
     const int64_t items = nblocks * NT2;
     const uint64_t pol_a = policy_evict_last();
-    const uint32_t b_full_l = cluster_addr(b_full, 0);
+    const uint32_t step_full_l = cluster_addr(step_full, 0);
     uint32_t nitem = 0;
-    RingPos bpos;
+    RingPos bpos, fill, lag;  // B data slot; step barrier of the fill; step the slot last held
     bool ok = true;
     // routing metadata of item w (its expert and the flat slots of this lane's 8 rows),
     // loaded one item ahead so the latency overlaps the current item's streaming
@@ -319,35 +326,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int row0 = pos0 + int(rank) * half;
       for (int kb = 0; kb < KT; ++kb) {
         const uint32_t s = bpos.slot;
-        // the slot's previous fill (one lap ago, opposite phase) must have been consumed
-        if (bpos.count >= uint32_t(BS) && !mbar_wait(&b_empty[s], bpos.phase ^ 1u, abort_v, p.status)) {
-          ok = false;
-          break;
+        // the slot's previous fill (BS steps ago) must have been consumed
+        if (bpos.count >= uint32_t(BS)) {
+          if (!mbar_wait(&step_empty[lag.slot], lag.phase, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          lag.next(DS);
         }
         if (lane == 0) {
           // rank 0 expects the bytes of both halves; each CTA copies its own half
-          if (leader) mbar_arrive_expect_tx(&b_full[s], uint32_t(nmma) * 128u * kBChunks);
-          tma_box3d_pair(sbase + p.rings.off_b + s * b_stage_bytes, map, row0, kb * kBChunks, b_full_l + s * 8u,
-                         pol_a);
+          if (leader) mbar_arrive_expect_tx(&step_full[fill.slot], uint32_t(nmma) * 128u * kBChunks);
+          tma_box3d_pair(sbase + p.rings.off_b + s * b_stage_bytes, map, row0, kb * kBChunks,
+                         step_full_l + fill.slot * 8u, pol_a);
         }
         bpos.next(BS);
+        fill.next(DS);
       }
       __syncwarp();
     }
-    // drain: rank 0 waits (bounded, ignoring abort) for the last min(BS, fills) fills of
-    // the B ring (both halves complete on its barriers), walking back from the current slot
+    // drain: rank 0 waits (bounded, ignoring abort) for the steps of the last min(BS,
+    // fills) fills (both halves complete on its barriers), walking back from the current one
     if (lane == 0 && leader) {
       int dummy = 0;
-      RingPos back = bpos;
-      const uint32_t n_back = bpos.count < uint32_t(BS) ? bpos.count : uint32_t(BS);
+      RingPos back = fill;
+      const uint32_t n_back = fill.count < uint32_t(BS) ? fill.count : uint32_t(BS);
       for (uint32_t i = 0; i < n_back; ++i) {
         if (back.slot == 0) {
-          back.slot = BS - 1;
+          back.slot = DS - 1;
           back.phase ^= 1u;
         } else {
           --back.slot;
         }
-        mbar_wait(&b_full[back.slot], back.phase, &dummy, p.status);
+        mbar_wait(&step_full[back.slot], back.phase, &dummy, p.status);
       }
     }
   } else if (warp == 2) {
@@ -395,7 +406,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
     if (leader && lane == 0) {
-      RingPos apos, bpos;
+      RingPos apos, bpos, step;
       uint64_t* last_bar = nullptr;
       uint32_t last_parity = 0;
       for (uint32_t it = 0;; ++it) {
@@ -410,35 +421,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t d_tmem = tmem_base + buf * 256;
         const int nmma = (d.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_m256(nmma);
-        const uint32_t chunk_bytes = uint32_t(nmma >> 1) * 128u;  // one chunk of this CTA's rows
+        // descriptor increments: the start-address field holds address / 16
+        const uint64_t b_chunk_inc = uint64_t(nmma >> 1) * 128u / 16u;  // one chunk of this CTA's rows
+        const uint64_t a_half_inc = uint64_t(kAHalfBytes) / 16u;
         bool ok = true;
-        for (int kb = 0; kb < KT && ok; ++kb) {
-          const uint32_t sb = bpos.slot, pb = bpos.phase;
-          if (!mbar_wait(&b_full[sb], pb, abort_v, p.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sa = apos.slot, pa = apos.phase;
-          if (!mbar_wait(&a_full[sa], pa, abort_v, p.status)) {
+        for (int kb = 0; kb < KT; ++kb) {
+          if (!mbar_wait(&step_full[step.slot], step.phase, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = sbase + p.rings.off_b + sb * b_stage_bytes;
-          const uint32_t a_addr = sbase + p.rings.off_a + sa * kAStageBytes;
+          const uint64_t ad = sw128_kmajor_desc(sbase + p.rings.off_a + apos.slot * kAStageBytes);
+          const uint64_t bd = sw128_kmajor_desc(sbase + p.rings.off_b + bpos.slot * b_stage_bytes);
 #pragma unroll
           for (int h = 0; h < kBChunks; ++h) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              tc2_mma(d_tmem, sw128_kmajor_desc(a_addr + h * kAHalfBytes + k * 32),
-                      sw128_kmajor_desc(b_addr + h * chunk_bytes + k * 32), idesc,
+              tc2_mma(d_tmem, ad + h * a_half_inc + k * 2, bd + h * b_chunk_inc + k * 2, idesc,
                       (kb > 0 || h > 0 || k > 0) ? 1u : 0u);
           }
-          tc2_commit_both(&a_empty[sa]);
+          tc2_commit_both(&step_empty[step.slot]);
+          last_bar = &step_empty[step.slot];
+          last_parity = step.phase;
+          step.next(DS);
           apos.next(AS);
-          tc2_commit_both(&b_empty[sb]);
-          last_bar = &b_empty[sb];
-          last_parity = pb;
           bpos.next(BS);
         }
         if (!ok) break;
@@ -456,9 +462,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int rb = w >> 1, hrow = w & 1;          // 16-row block, upper or lower 8 rows
     const int g = lane >> 2, t = lane & 3;
     const int row = rb * 16 + 8 * hrow + g;
-    const uint32_t a_full_l = cluster_addr(a_full, 0);
+    const uint32_t step_full_l = cluster_addr(step_full, 0);
     uint32_t rstage = 0;
-    RingPos apos;
+    RingPos apos, fill, lag;  // A data slot; step barrier of the fill; step the slot last held
     for (uint32_t it = 0;; ++it) {
       const uint32_t ds = it % kDescRingTC;
       if (!mbar_wait(&dfull[ds], (it / kDescRingTC) & 1, abort_v, p.status)) break;
@@ -478,17 +484,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint4 c = lds128(tb + rb * 1024 + hrow * 512 + g * 64 + t * 16);
           const uint2 sc = lds64(tb + kTileCodeBytes + rb * 128 + g * 16 + hrow * 8);
           const uint32_t s = apos.slot;
-          if (apos.count >= uint32_t(AS) && !mbar_wait(&a_empty[s], apos.phase ^ 1u, abort_v, p.status)) {
-            ok = false;
-            break;
+          // the slot's previous fill (AS steps ago) must have been consumed
+          if (apos.count >= uint32_t(AS)) {
+            if (!mbar_wait(&step_empty[lag.slot], lag.phase, abort_v, p.status)) {
+              ok = false;
+              break;
+            }
+            lag.next(DS);
           }
           const uint32_t a_stage = sbase + p.rings.off_a + s * kAStageBytes;
           dequant_row_half<0>(c, sc.x, a_stage, row, g, t);
           dequant_row_half<1>(c, sc.y, a_stage + kAHalfBytes, row, g, t);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(a_full_l + s * 8u);
+          if (lane == 0) mbar_arrive_cluster(step_full_l + fill.slot * 8u);
           apos.next(AS);
+          fill.next(DS);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&raw_empty[rs]);
