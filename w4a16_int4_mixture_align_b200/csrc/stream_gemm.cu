@@ -6,21 +6,22 @@
 // indexierter Decode"); the same operand orientation is used here, on sm_100a, with the
 // weight tiles streamed by bulk asynchronous copies through a deep shared-memory ring:
 //
-//   warp 0        producer: per item (routing block b, token chunk c, 128-row tile nt)
-//                 it publishes a descriptor, then per stage of KTS consecutive 128-wide
-//                 K tiles issues ONE bulk copy of their codes + scales (up to 36 KiB:
-//                 a bulk copy has a high fixed cost, so bytes per copy decide the
-//                 streaming rate). The few routed activation rows are small and shared
-//                 by every warp, so consumers read them straight from global memory
-//                 through L1 (ld.global.nc) instead of staging them.
-//   warps 1..8    consumer group 0, warps 9..16 group 1: group g takes the tiles of
-//                 parity g inside each stage; warp w owns 16 physical rows. Codes go
-//                 shared -> registers and dequantise to bf16 pairs (subtract 8, then
-//                 scale) that are exactly the A fragments of mma.m16n8k16; tokens are N.
-//   epilogue      group 1 hands its partial sums to group 0, which adds them and applies
-//                 SiLU(gate)*up (gate_up; gate and up rows are interleaved by the repack)
-//                 or writes the expert output (down) to the per-slot buffer y, which the
-//                 combine weights and sums.
+//   warp 0        producer: takes the work items (routing block b, token chunk c, 128-row
+//                 tile nt) two at a time, publishes both descriptors, then streams the two
+//                 items' stages alternately, each stage ONE bulk copy of KTS consecutive
+//                 128-wide K tiles (codes + scales, up to 36 KiB: a bulk copy has a high fixed
+//                 cost, so bytes per copy decide the streaming rate). The few routed
+//                 activation rows are small and shared by every warp, so consumers read them
+//                 straight from global memory through L1 (ld.global.nc) instead of staging them.
+//   warps 1..8    consumer group 0 takes the first item of each pair, warps 9..16 group 1
+//                 the second; a warp owns 16 physical rows and consumes every tile of its
+//                 item's stages. Codes go shared -> registers and dequantise to bf16 pairs
+//                 (subtract 8, then scale) that are exactly the A fragments of mma.m16n8k16;
+//                 tokens are N. Each group then runs its own epilogue: SiLU(gate)*up (gate_up;
+//                 gate and up rows are interleaved by the repack) or the expert output (down)
+//                 to the per-slot buffer y, which the combine weights and sums. Whole items per
+//                 group need no hand-over of partial sums between the groups, which matters
+//                 when K is short and an item is a single stage.
 //
 // Every wait is an mbarrier wait bounded in time; on timeout the CTA raises
 // CHORD_DEV_TIMEOUT, unwinds, and the producer waits (bounded) for its copies in flight.
@@ -59,6 +60,9 @@ struct StreamParams {
 
 struct ItemDesc {
   int e, nt, pos0, end;     // end = 1 marks the end of the item sequence
+  uint32_t s0;              // global index of the item's first stage
+  int sstride;              // 2 when its stages alternate with the paired item's, else 1
+  int pad[2];
   int f[kMaxTC];            // flat slot of each token column, -1 when padding
 };
 
@@ -66,13 +70,10 @@ template <int TC>
 struct Smem {
   static constexpr int kKTS = 4;                                // K tiles per stage
   static constexpr int kStageBytes = kKTS * kTileBytes;
-  static constexpr int kHandoverBytes = 8 * 32 * (TC / 8) * 4 * 4;  // 8 warps x 32 lanes x 4*NT floats
   static constexpr int kBudget = 200 * 1024;
-  static constexpr int kFit =
-      (kBudget - kHandoverBytes - kDescRing * int(sizeof(ItemDesc)) - 1024) / kStageBytes;
+  static constexpr int kFit = (kBudget - kDescRing * int(sizeof(ItemDesc)) - 1024) / kStageBytes;
   static constexpr int kStages = kFit > 12 ? 12 : kFit;
-  static constexpr int kBytes =
-      kStages * kStageBytes + kHandoverBytes + kDescRing * int(sizeof(ItemDesc)) + 1024;
+  static constexpr int kBytes = kStages * kStageBytes + kDescRing * int(sizeof(ItemDesc)) + 1024;
 };
 
 __device__ __forceinline__ uint4 ldg_nc128(const void* p) {
@@ -88,7 +89,7 @@ __device__ __forceinline__ uint4 ldg_nc128(const void* p) {
 template <int NT8, int NSET, int NTILE, class S>
 __device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb, int lane,
                                               const uint16_t* const (&xrow)[NT8],
-                                              float (&acc)[NT8][NSET][4]) {
+                                              float (&acc)[NT8][NSET][4], int chain0) {
   const int g = lane >> 2, t = lane & 3;
   uint4 c0[NTILE], c1[NTILE], sv[NTILE];
 #pragma unroll
@@ -123,8 +124,8 @@ __device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb
       const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
 #pragma unroll
       for (int n8 = 0; n8 < NT8; ++n8) {
-        mma_bf16_16816(acc[n8][(2 * u) % NSET], a_lo, xv[u][j][n8].x, xv[u][j][n8].y);
-        mma_bf16_16816(acc[n8][(2 * u + 1) % NSET], a_hi, xv[u][j][n8].z, xv[u][j][n8].w);
+        mma_bf16_16816(acc[n8][(chain0 + 2 * u) % NSET], a_lo, xv[u][j][n8].x, xv[u][j][n8].y);
+        mma_bf16_16816(acc[n8][(chain0 + 2 * u + 1) % NSET], a_hi, xv[u][j][n8].z, xv[u][j][n8].w);
       }
     }
   }
@@ -139,16 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
   static_assert(NSTAGE >= 3 && NSTAGE < kDescRing, "stage count");
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stages = smem;
-  float* handover = reinterpret_cast<float*>(smem + NSTAGE * S::kStageBytes);
-  ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + NSTAGE * S::kStageBytes + S::kHandoverBytes);
+  ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + NSTAGE * S::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(descs) +
                                                kDescRing * sizeof(ItemDesc));
   uint64_t* full = bars;                        // [NSTAGE]
-  uint64_t* empty = full + NSTAGE;              // [NSTAGE]
+  uint64_t* empty = full + NSTAGE;              // [NSTAGE] the owning group's 8 warps
   uint64_t* dfull = empty + NSTAGE;             // [kDescRing]
-  uint64_t* dempty = dfull + kDescRing;         // [kDescRing]
-  uint64_t* hfull = dempty + kDescRing;         // [1] group 1 -> group 0
-  uint64_t* hempty = hfull + 1;                 // [1] group 0 -> group 1
+  uint64_t* dempty = dfull + kDescRing;         // [kDescRing] the owning group's 8 warps
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -162,14 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     }
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], 8);
     }
     for (int s = 0; s < kDescRing; ++s) {
       mbar_init(&dfull[s], 1);
       mbar_init(&dempty[s], 8);
     }
-    mbar_init(hfull, 8);
-    mbar_init(hempty, 8);
     fence_barrier_init();
   }
   __syncthreads();
@@ -191,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     const uint64_t pol_w = policy_evict_first();
     uint32_t stage = 0;      // global stage counter
     uint32_t nitem = 0;      // published descriptors
+    bool ok = true;
     // routing metadata of item w: its expert and this lane's flat slot (lane < TC). The
     // loads run kLook items ahead (a small register queue) so their latency overlaps
     // the streaming of earlier items instead of stalling at every item boundary.
@@ -211,56 +208,78 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     int qe[kLook], qpos[kLook], qf[kLook];
 #pragma unroll
     for (int i = 0; i < kLook; ++i) load_meta(blockIdx.x + int64_t(i) * gridDim.x, qe[i], qpos[i], qf[i]);
-    for (int64_t w = blockIdx.x;; w += gridDim.x) {
-      const bool end = w >= items;
-      int e = qe[0], pos0 = qpos[0], fval = qf[0];
-      const int nt = end ? 0 : int(w % NTILES);
+    int64_t w_next = blockIdx.x;
+    // the next item with at least one routed row, or false at the end
+    auto pop_item = [&](int& e, int& nt, int& pos0, int& fval) -> bool {
+      while (w_next < items) {
+        const int64_t w = w_next;
+        w_next += gridDim.x;
+        e = qe[0];
+        pos0 = qpos[0];
+        fval = qf[0];
+        nt = int(w % NTILES);
 #pragma unroll
-      for (int i = 0; i + 1 < kLook; ++i) {
-        qe[i] = qe[i + 1];
-        qpos[i] = qpos[i + 1];
-        qf[i] = qf[i + 1];
-      }
-      load_meta(w + int64_t(kLook) * gridDim.x, qe[kLook - 1], qpos[kLook - 1], qf[kLook - 1]);
-      if (!end) {
+        for (int i = 0; i + 1 < kLook; ++i) {
+          qe[i] = qe[i + 1];
+          qpos[i] = qpos[i + 1];
+          qf[i] = qf[i + 1];
+        }
+        load_meta(w + int64_t(kLook) * gridDim.x, qe[kLook - 1], qpos[kLook - 1], qf[kLook - 1]);
         if (!(fval >= 0 && fval < p.n_slots) || unsigned(e) >= unsigned(p.E)) fval = -1;
-        if (__ballot_sync(0xffffffffu, fval >= 0) == 0) continue;  // nothing routed here
+        if (__ballot_sync(0xffffffffu, fval >= 0) != 0) return true;  // something routed here
       }
-      // publish the item (or the end marker) to the consumers
+      return false;
+    };
+    // publishes one descriptor (or an end marker) at index nitem
+    auto publish = [&](int e, int nt, int pos0, int fval, bool end, uint32_t s0, int sstride) -> bool {
       const uint32_t ds = nitem % kDescRing;
       if (nitem >= kDescRing &&
           !mbar_wait(&dempty[ds], ((nitem / kDescRing) - 1) & 1, abort_v, p.status))
-        break;
+        return false;
       ItemDesc* d = &descs[ds];
       if (lane < TC) d->f[lane] = fval;
       if (lane == 0) {
-        d->e = e; d->nt = nt; d->pos0 = pos0; d->end = end ? 1 : 0;
+        d->e = e; d->nt = nt; d->pos0 = pos0; d->end = end ? 1 : 0; d->s0 = s0; d->sstride = sstride;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&dfull[ds]);
       ++nitem;
-      if (end) break;
-      // stream the item: one bulk copy of KTS tiles (codes + scales) per stage
-      const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
-      bool ok = true;
-      for (int ks = 0; ks < KS; ++ks, ++stage) {
-        const uint32_t slot = stage % NSTAGE;
-        if (stage >= uint32_t(NSTAGE) &&
-            !mbar_wait(&empty[slot], ((stage / NSTAGE) - 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        const int kt0 = ks * KTS;
-        const int ntl = min(KTS, KT - kt0);
-        if (lane == 0) {
-          uint8_t* st = stages + slot * S::kStageBytes;
-          mbar_arrive_expect_tx(&full[slot], uint32_t(ntl) * kTileBytes);
-          bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &full[slot],
-                        pol_w);
-        }
+      return true;
+    };
+    // streams stage ks of the item on expert e, tile nt: one bulk copy of up to KTS tiles
+    auto stream_stage = [&](int e, int nt, int ks) -> bool {
+      const uint32_t slot = stage % NSTAGE;
+      if (stage >= uint32_t(NSTAGE) &&
+          !mbar_wait(&empty[slot], ((stage / NSTAGE) - 1) & 1, abort_v, p.status))
+        return false;
+      const int kt0 = ks * KTS;
+      const int ntl = min(KTS, KT - kt0);
+      if (lane == 0) {
+        uint8_t* st = stages + slot * S::kStageBytes;
+        const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
+        mbar_arrive_expect_tx(&full[slot], uint32_t(ntl) * kTileBytes);
+        bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &full[slot], pol_w);
       }
-      if (!ok) break;
+      ++stage;
+      return true;
+    };
+    // items two at a time: group 0 takes the first, group 1 the second; their stages
+    // alternate in the ring so both groups stream concurrently
+    while (ok) {
+      int ea, nta, pa, fa, eb, ntb, pb, fb;
+      if (!pop_item(ea, nta, pa, fa)) break;
+      const bool has_b = pop_item(eb, ntb, pb, fb);
+      ok = publish(ea, nta, pa, fa, false, stage, has_b ? 2 : 1);
+      if (ok && has_b) ok = publish(eb, ntb, pb, fb, false, stage + 1, 2);
+      for (int ks = 0; ks < KS && ok; ++ks) {
+        ok = stream_stage(ea, nta, ks);
+        if (ok && has_b) ok = stream_stage(eb, ntb, ks);
+      }
+      if (!has_b) break;
     }
+    // end markers at two consecutive indices: one reaches each group
+    if (ok) ok = publish(0, 0, 0, -1, true, 0, 1);
+    if (ok) publish(0, 0, 0, -1, true, 0, 1);
     // drain: wait (bounded, ignoring the abort flag) for every copy still in flight
     if (lane == 0) {
       int dummy = 0;
@@ -273,11 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 
   // ------------------------------------------------------------------ consumers
   const int cw = warp - 1;             // 0..15
-  const int grp = cw >> 3;             // 0 or 1
+  const int grp = cw >> 3;             // 0 or 1: the first or second item of each pair
   const int rb = cw & 7;               // 16-row block inside the tile
   const int g = lane >> 2, t = lane & 3;
-  uint32_t stage0 = 0;                 // stage counter at the item's first K step
-  for (uint32_t it = 0;; ++it) {
+  for (uint32_t it = grp;; it += 2) {
     const uint32_t ds = it % kDescRing;
     if (!mbar_wait(&dfull[ds], (it / kDescRing) & 1, abort_v, p.status)) return;
     const ItemDesc& d = descs[ds];
@@ -299,8 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 #pragma unroll
       for (int q = 0; q < NSET; ++q) acc[i][q][0] = acc[i][q][1] = acc[i][q][2] = acc[i][q][3] = 0.f;
 
+    const uint32_t s0 = d.s0;
+    const int sstride = d.sstride;
     for (int ks = 0; ks < KS; ++ks) {
-      const uint32_t s = stage0 + ks;
+      const uint32_t s = s0 + uint32_t(ks * sstride);
       const uint32_t slot = s % NSTAGE;
       if (!mbar_wait(&full[slot], (s / NSTAGE) & 1, abort_v, p.status)) return;
       const int ntl = min(KTS, KT - ks * KTS);
@@ -310,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       const uint16_t* xrow[NT8];
 #pragma unroll
       for (int n8 = 0; n8 < NT8; ++n8) xrow[n8] = xrow0[n8] + ks * KTS * kTileK;
-      for (int i = grp; i < ntl; i += 2) consume_tiles<NT8, NSET, 1, S>(stg, i, rb, lane, xrow, acc);
+      for (int i = 0; i < ntl; ++i) consume_tiles<NT8, NSET, 1, S>(stg, i, rb, lane, xrow, acc, (i & 1) * 2);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
@@ -324,28 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
         for (int q = 0; q < NSET; ++q) v += acc[i][q][c];
         accs[i][c] = v;
       }
-    stage0 += KS;
 
-    // ---- hand over and epilogue
-    float* hw = handover + (rb * 32 + lane) * (4 * NT8);
-    if (grp == 1) {
-      if (it > 0 && !mbar_wait(hempty, (it - 1) & 1, abort_v, p.status)) return;
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8)
-        *reinterpret_cast<float4*>(hw + 4 * n8) = make_float4(accs[n8][0], accs[n8][1], accs[n8][2], accs[n8][3]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(hfull);
-      continue;
-    }
-    if (!mbar_wait(hfull, it & 1, abort_v, p.status)) return;
-#pragma unroll
-    for (int n8 = 0; n8 < NT8; ++n8) {
-      const float4 o = *reinterpret_cast<const float4*>(hw + 4 * n8);
-      accs[n8][0] += o.x; accs[n8][1] += o.y; accs[n8][2] += o.z; accs[n8][3] += o.w;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(hempty);
-
+    // ---- epilogue (this group's item)
     if (EPI == kGateUp) {
       const int i_col = d.nt * (kTileN / 2) + rb * 8 + g;  // intermediate column
 #pragma unroll
