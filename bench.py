@@ -187,7 +187,9 @@ def run_chord(args, rank, world, local_rank):
     ids = torch.from_numpy(ids_np).to(dev)
     tw = torch.from_numpy(tw_np).to(dev)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
+    # all GPU work of the timed leg runs on one side stream (graph capture needs one)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
 
     def step():
         layer.forward(x, ids, tw, out=out)
@@ -199,10 +201,28 @@ def run_chord(args, rank, world, local_rank):
     assert layer.check_status() == 0
 
     # per-kernel events: [start, align done, gate_up done, down done, combine done] per step
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(K)]
     for row in ev:
         for e in row:
             e.record(stream)
+    torch.cuda.synchronize()
+
+    # The K timed steps are captured once into a CUDA graph (the library enqueues
+    # everything on the caller's stream and never reads back, so a step is capturable),
+    # then replayed: the timed region runs exactly the K steps' kernels, without the host
+    # launch gaps of an eager loop. The per-kernel events are captured with them.
+    launches0 = chord.chord_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for k in range(K):
+            ev[k][0].record(stream)
+            layer.align(ids)
+            chord.chord_set_timing_events(ev[k][1:5])
+            chord.chord_moe_forward(x, ids, tw, layer.sorted_ids, layer.expert_ids, layer.ntp, layer.block_m,
+                                    layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace)
+            chord.chord_set_timing_events(None)
+    launches = chord.chord_launch_count() - launches0  # kernels per replay (captured once)
+    graph.replay()  # one untimed replay
     torch.cuda.synchronize()
 
     visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
@@ -211,24 +231,17 @@ def run_chord(args, rank, world, local_rank):
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
-    launches0 = chord.chord_launch_count()
     t_wall0 = time.time()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for k in range(K):
-        ev[k][0].record(stream)
-        layer.align(ids)
-        chord.chord_set_timing_events(ev[k][1:5])
-        chord.chord_moe_forward(x, ids, tw, layer.sorted_ids, layer.expert_ids, layer.ntp, layer.block_m,
-                                layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace)
-        chord.chord_set_timing_events(None)
+    graph.replay()
     stop.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
     barrier(world)
-    launches = chord.chord_launch_count() - launches0
     elapsed_ms = start.elapsed_time(stop)
     assert layer.check_status() == 0
+    del graph
 
     seg = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in range(K)])
     seg_ms = seg.mean(axis=0)  # align, gate_up, down, combine

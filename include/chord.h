@@ -231,7 +231,8 @@ CHORD_API chord_status_t chord_moe_check_status(void* workspace, chord_stream_t 
  * calling thread records the caller-owned cudaEvent_t handles events[0..3] on its
  * stream: [0] right before the gate_up GEMM kernel (after routing validation and, on
  * the tensor-core schedule, the row permutation), [1] between the gate_up and down GEMM
- * kernels, [2] after the down GEMM, [3] after the combine. n == 0 clears the hook. The handles must stay
+ * kernels, [2] after the down GEMM, [3] after the combine. Records use cudaEventRecordExternal,
+ * so a forward captured into a CUDA graph records them when the graph is replayed. n == 0 clears the hook. The handles must stay
  * valid while set. Returns CHORD_ERR_INVALID_ARG for other n or null handles.
  *
  * chord_launch_count: number of CUDA kernels this library has launched in the process

@@ -338,10 +338,10 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   cudaEvent_t mid = timing ? g_timing[1] : nullptr;
   err = tensor ? launch_tc_gemms(a, stream, first, mid) : launch_stream_gemms(a, stream, first, mid);
   if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");
-  if (timing && (err = cudaEventRecord(g_timing[2], stream)) != cudaSuccess)
+  if (timing && (err = record_timing_event(g_timing[2], stream)) != cudaSuccess)
     return cuda_fail(err, "timing event");
   if ((err = launch_combine(a, stream)) != cudaSuccess) return cuda_fail(err, "combine launch");
-  if (timing && (err = cudaEventRecord(g_timing[3], stream)) != cudaSuccess)
+  if (timing && (err = record_timing_event(g_timing[3], stream)) != cudaSuccess)
     return cuda_fail(err, "timing event");
   return CHORD_OK;
 }

@@ -333,6 +333,13 @@ void count_launches(int n);
 
 // `mid` (may be null) is recorded on the stream between the gate_up and down GEMMs.
 cudaError_t launch_validate(const ForwardArgs& a, cudaStream_t stream);
+// Records a caller's timing event on `stream`. Under stream capture the record becomes an
+// event node of the graph (a plain record would only order the capture), so a captured
+// forward still times its kernels when the graph is replayed.
+inline cudaError_t record_timing_event(cudaEvent_t ev, cudaStream_t stream) {
+  return cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+}
+
 // `first` (if set) is recorded right before the gate_up GEMM kernel, `mid` between the two
 // GEMM kernels.
 cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid);

@@ -429,11 +429,11 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
   p.role = CHORD_ROLE_GATE_UP;
   p.act = a.x;
   p.act_ld = a.H;
-  cudaError_t err = first ? cudaEventRecord(first, stream) : cudaSuccess;
+  cudaError_t err = first ? record_timing_event(first, stream) : cudaSuccess;
   if (err != cudaSuccess) return err;
   err = launch_tc<kGateUp>(p, tc, grid, stream);
   if (err != cudaSuccess) return err;
-  if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
+  if (mid && (err = record_timing_event(mid, stream)) != cudaSuccess) return err;
 
   // down: W2 [E, H, I], activations a [cap, I]
   p.blob = a.w2;

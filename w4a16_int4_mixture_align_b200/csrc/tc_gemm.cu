@@ -743,9 +743,9 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
   p.N = 2 * a.I;
   p.K = a.H;
   p.role = CHORD_ROLE_GATE_UP;
-  if (first && (err = cudaEventRecord(first, stream)) != cudaSuccess) return err;
+  if (first && (err = record_timing_event(first, stream)) != cudaSuccess) return err;
   if ((err = launch_one<kGateUp>(maps, p, grid, stream)) != cudaSuccess) return err;
-  if (mid && (err = cudaEventRecord(mid, stream)) != cudaSuccess) return err;
+  if (mid && (err = record_timing_event(mid, stream)) != cudaSuccess) return err;
 
   // down: W2 [E, H, I]; B rows of the K-blocked intermediate a, already in routing order
   if ((err = box_maps(&maps, a.a, a.cap, a.I)) != cudaSuccess) return err;
