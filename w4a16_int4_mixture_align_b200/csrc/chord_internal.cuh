@@ -83,13 +83,12 @@ __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1
 // ------------------------------------------------------------------------------------
 // Workspace of chord_moe_forward:
 //   [status 256 B][a: cap x I bf16][y: cap x H fp32][xs: cap x H bf16][slot_pos: T*topk i32]
-// a is the SiLU*up intermediate by sorted position (row-major [cap, I] on the streaming
-// schedule, K-blocked [I/64][cap][64] on the tensor-core schedule); y the expert outputs
+// a is the SiLU*up intermediate by sorted position (row-major [cap, I]); y the expert outputs
 // before the top-k weight (by flat slot [T*topk, H] on the streaming schedule, by sorted
 // position in 128-column blocks [H/128][cap][128] on the tensor-core schedule, so that a
-// work item writes one contiguous block); xs the hidden rows in sorted order, K-blocked
-// [H/64][cap][64], and slot_pos the sorted position of every local flat slot (both
-// tensor-core schedule only).
+// work item writes one contiguous block); xs the hidden rows in sorted order [cap, H],
+// and slot_pos the sorted position of every local flat slot (both tensor-core schedule
+// only).
 struct ForwardWorkspace {
   uint64_t a_offset, y_offset, xs_offset, slot_pos_offset, total;
 };
@@ -315,10 +314,10 @@ struct ForwardArgs {
   const uint8_t* w13;
   const uint8_t* w2;
   uint16_t* out;
-  uint16_t* a;     // bf16 intermediate by sorted position: [cap, I], or [I/64][cap][64] (tensor core)
+  uint16_t* a;     // [cap, I] bf16 intermediate by sorted position
   float* y;        // fp32 expert outputs before the top-k weight: [T*topk, H] by flat slot, or
                    // [H/128][cap][128] by sorted position (y_blocked, tensor core)
-  uint16_t* xs;    // [H/64][cap][64] bf16 hidden rows in sorted order (tensor-core schedule)
+  uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
   int32_t* slot_pos;  // [T*topk] sorted position of each local flat slot (tensor-core schedule)
   bool y_blocked;     // y is by sorted position in 128-column blocks
   uint32_t* status;
@@ -344,7 +343,7 @@ inline cudaError_t record_timing_event(cudaEvent_t ev, cudaStream_t stream) {
 // GEMM kernels.
 cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid);
 cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent_t first, cudaEvent_t mid);
-// xs <- the hidden rows in routing order, K-blocked [H/64][cap][64] (tensor-core schedule).
+// xs <- the hidden rows in routing order [cap, H] (tensor-core schedule).
 cudaError_t launch_permute_rows(const ForwardArgs& a, cudaStream_t stream);
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream);
 

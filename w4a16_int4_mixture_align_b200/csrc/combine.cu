@@ -126,7 +126,7 @@ __global__ void validate_kernel(const int32_t* __restrict__ topk_ids,
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
   int64_t grid = a.T * ((a.H + kCombineCols - 1) / kCombineCols);
-  if (grid > int64_t(a.num_sms) * 16) grid = int64_t(a.num_sms) * 16;
+  if (grid > int64_t(a.num_sms) * 64) grid = int64_t(a.num_sms) * 64;
   if (a.y_blocked)
     combine_kernel<true><<<unsigned(grid), kCombineThreads, 0, stream>>>(
         a.topk_ids, a.topk_weights, a.y, a.slot_pos, a.out, a.T, a.H, a.topk, a.E, a.cap);

@@ -2,17 +2,15 @@
 //
 // The tensor-core GEMMs read the activation operand as whole tiles of consecutive rows
 // (one TMA box per 128-K step), so the hidden states are copied once into the order of
-// sorted_ids (the routing sort of the Chord blog's indexed path), K-blocked as
-// [H/64][cap][64]: xs[c / 64][pos][c % 64] = x[sorted_ids[pos] / topk][c]. Padding
-// positions (sentinel slots) are skipped; the GEMMs never read them back into a result.
+// sorted_ids (the routing sort of the Chord blog's indexed path), row-major:
+// xs[pos][c] = x[sorted_ids[pos] / topk][c]. Padding positions (sentinel slots) are
+// skipped; the GEMMs never read them back into a result.
 // The same pass records slot_pos[f] = pos, the inverse of sorted_ids over the local
 // slots, with which the combine finds a slot's expert output in the position-ordered y.
 //
-// One warp copies one routed row: 32 lanes read 512 contiguous bytes of the source row
-// per step and write them as four 128-byte runs, one per 64-column chunk. A hidden row is
+// One warp copies one routed row, 512 contiguous bytes per step each way. A hidden row is
 // read once per local slot of its token (up to top-k times), so the reads ask L2 to keep
-// it (evict_last) while the copies, larger than L2, stream out (evict_first). (Staging 32
-// rows in shared memory to write 4 KiB runs measured slower: fewer CTAs and two phases.)
+// it (evict_last) while the copies, larger than L2, stream out (evict_first).
 #include "chord_internal.cuh"
 
 namespace chord {
@@ -49,12 +47,8 @@ __global__ void __launch_bounds__(32 * kPermuteWarps) permute_rows_kernel(
     if (f < 0 || f >= n_slots) continue;
     if (lane == 0) slot_pos[f] = int32_t(pos);
     const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(f / topk) * H);
-    uint16_t* dst = xs + pos * 64;
-    for (int v = lane; v < vec; v += 32) {
-      const uint4 val = ldg_keep(src + v, keep);
-      const int c = v * 8;
-      stg_stream(dst + int64_t(c >> 6) * cap * 64 + (c & 63), val, stream);
-    }
+    uint4* dst = reinterpret_cast<uint4*>(xs + pos * H);
+    for (int v = lane; v < vec; v += 32) stg_stream(dst + v, ldg_keep(src + v, keep), stream);
   }
 }
 

@@ -18,8 +18,8 @@
 //
 //   warp 0      activation producer (both CTAs): per 128-wide K step one TMA request
 //               for this CTA's half of the block's rows, two 64-column chunks of them
-//               (a 3-D box of the K-blocked activation layout [K/64][rows][64], 128-byte
-//               swizzle), into its B ring; the copies of both CTAs complete on the B
+//               (a 3-D box over the row-major activations viewed as {64 columns, rows,
+//               chunks}, 128-byte swizzle, landing chunk-major), into its B ring; the copies of both CTAs complete on the B
 //               barrier of rank 0. One request per step matters: each TMA issue holds the
 //               issuing thread for a few hundred cycles, so the box height equals the
 //               half-block (a tensor map per height, 8..128 rows). The rows are contiguous
@@ -38,7 +38,7 @@
 //               the ring stages and publishes the accumulator.
 //   warps 19..26 epilogue (both CTAs, two per TMEM lane quadrant, alternate 16-column
 //               chunks): tcgen05.ld of this CTA's 128 accumulator rows; SiLU(gate)*up
-//               written to the K-blocked bf16 intermediate (gate_up), or the fp32 expert
+//               written to the bf16 intermediate (gate_up), or the fp32 expert
 //               output written by sorted position in 128-column blocks (down; the combine
 //               applies the top-k weight).
 //               Double buffering lets it overlap the next item.
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float u = __shfl_down_sync(0xffffffffu, v[c], 8);
               const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
               if (gate && f >= 0)
-                p.a_out[(int64_t(i_col >> 6) * p.cap + d.pos0 + c0 + c) * 64 + (i_col & 63)] =
+                p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
             }
           } else {
@@ -608,8 +608,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Box maps of a K-blocked bf16 tensor [K/64][rows][64]: map i has box {64 columns,
-// 8 * (i + 1) rows, kBChunks chunks}, 128-byte swizzle; rows past the end read as zero.
+// Box maps of a row-major bf16 tensor [rows][K], viewed as 3-D {64 columns, rows,
+// K/64 chunks} with strides {K*2, 128} bytes, so that a box {64, R, kBChunks} lands in
+// shared memory chunk-major, [chunk][row][128 B]: the K-blocked tile the MMA reads. Map
+// i has R = 8 * (i + 1) rows, 128-byte swizzle; rows past the end read as zero.
 // Encoding sixteen maps costs host time, so the last few sets are kept, keyed by the
 // tensor's address and shape (the workspace of a layer is reused call after call).
 cudaError_t box_maps(BoxMaps* out, const void* base, int64_t rows, int K) {
@@ -634,7 +636,7 @@ cudaError_t box_maps(BoxMaps* out, const void* base, int64_t rows, int K) {
   if (!fn) return cudaErrorNotSupported;
   BoxMaps maps;
   cuuint64_t dims[3] = {64, cuuint64_t(rows), cuuint64_t(K / 64)};
-  cuuint64_t strides[2] = {128, cuuint64_t(rows) * 128};
+  cuuint64_t strides[2] = {cuuint64_t(K) * 2, 128};
   cuuint32_t estr[3] = {1, 1, 1};
   for (int i = 0; i < kNumBoxMaps; ++i) {
     cuuint32_t box[3] = {64, cuuint32_t(8 * (i + 1)), cuuint32_t(kBChunks)};
