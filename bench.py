@@ -299,10 +299,14 @@ def run_chord(args, rank, world, local_rank):
                     "traffic": recorded_traffic("stream_gemm_gate_up", args.workload),
                     "algorithmic_bytes_per_launch": work["gate_up_bytes"]}
     else:
+        # the GEMM is timed inside K back-to-back steps (hundreds of ms of tensor work under
+        # the power cap), so its denominator is the sustained cuBLAS figure; the burst
+        # fraction is reported beside it
         achieved = work["gate_up_flops"] / (gu_us * 1e-6) / 1e12
         roofline = {"bound": "tensor", "kernel": "gate_up GEMM", "achieved": round(achieved, 1),
-                    "peak": tf_burst, "unit": "TFLOP/s", "frac": round(achieved / tf_burst, 4),
-                    "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                    "peak": tf_sust, "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
+                    "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long run of steps)",
+                    "peak_burst": tf_burst, "frac_of_burst": round(achieved / tf_burst, 4),
                     "traffic": recorded_traffic("tc_gemm_gate_up", args.workload),
                     "algorithmic_flops_per_launch": work["gate_up_flops"]}
     layer_us = elapsed_ms * 1000.0 / K
