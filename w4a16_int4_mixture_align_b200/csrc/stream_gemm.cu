@@ -86,18 +86,30 @@ __device__ __forceinline__ uint4 ldg_nc128(const void* p) {
 // accumulates them against the routed activation rows (xrow[n8] points at this lane's row
 // of 8-token tile n8, advanced to the stage's first K): the A fragments of
 // mma.m16n8k16 come straight out of dequant8; tokens are the N dimension.
+// This warp's code words (rows g and g + 8 of its 16-row block) and scales of one tile.
+struct TileCodes {
+  uint4 c0, c1, sv;
+};
+__device__ __forceinline__ TileCodes load_tile_codes(const uint8_t* stg, int tile, int rb, int lane) {
+  const uint8_t* st = stg + tile * kTileBytes;
+  TileCodes tc;
+  tc.c0 = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
+  tc.c1 = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
+  tc.sv = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + (lane >> 2) * 16);
+  return tc;
+}
+
 template <int NT8, int NSET, int NTILE, class S>
-__device__ __forceinline__ void consume_tiles(const uint8_t* stg, int t0, int rb, int lane,
+__device__ __forceinline__ void consume_tiles(const TileCodes (&codes)[NTILE], int t0, int lane,
                                               const uint16_t* const (&xrow)[NT8],
                                               float (&acc)[NT8][NSET][4], int chain0) {
-  const int g = lane >> 2, t = lane & 3;
+  const int t = lane & 3;
   uint4 c0[NTILE], c1[NTILE], sv[NTILE];
 #pragma unroll
   for (int u = 0; u < NTILE; ++u) {
-    const uint8_t* st = stg + (t0 + 2 * u) * kTileBytes;
-    c0[u] = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
-    c1[u] = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
-    sv[u] = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + g * 16);
+    c0[u] = codes[u].c0;
+    c1[u] = codes[u].c1;
+    sv[u] = codes[u].sv;
   }
   // the tile's activation fragments, issued together ahead of the dequantisation so their
   // L1 latency overlaps it
@@ -330,7 +342,15 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       const uint16_t* xrow[NT8];
 #pragma unroll
       for (int n8 = 0; n8 < NT8; ++n8) xrow[n8] = xrow0[n8] + ks * KTS * kTileK;
-      for (int i = 0; i < ntl; ++i) consume_tiles<NT8, NSET, 1, S>(stg, i, rb, lane, xrow, acc, (i & 1) * 2);
+      // software-pipelined over the stage's tiles: tile i + 1's codes are loaded from shared
+      // memory before tile i is dequantised, so their latency overlaps the math
+      TileCodes cur[1] = {load_tile_codes(stg, 0, rb, lane)};
+      for (int i = 0; i < ntl; ++i) {
+        TileCodes nxt = cur[0];
+        if (i + 1 < ntl) nxt = load_tile_codes(stg, i + 1, rb, lane);
+        consume_tiles<NT8, NSET, 1, S>(cur, i, lane, xrow, acc, (i & 1) * 2);
+        cur[0] = nxt;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
