@@ -49,6 +49,9 @@ def _load():
         lib.oracle_align_blocks.argtypes = [i64, i64, i64, i64]
         lib.oracle_align_blocks.restype = i64
         lib.oracle_moe_align.argtypes = [i32p, i64, i64, i64, i64, i32p, i32p, i32p, i32p]
+        lib.oracle_grouped_gemm.restype = ctypes.c_int
+        lib.oracle_grouped_gemm.argtypes = [u16p, i64, i64, i32p, u16p, i64, i64, i32p, i32p, i64, u16p,
+                                            ctypes.c_int]
         lib.oracle_router_topk.restype = ctypes.c_int
         lib.oracle_router_topk.argtypes = [f32p, i64, i64, i64, i32p, f32p]
         lib.oracle_moe_align.restype = ctypes.c_int
@@ -108,6 +111,34 @@ def moe_align(topk_ids: np.ndarray, E: int, block_m: int):
     if rc != 0:
         raise ValueError(f"oracle_moe_align failed ({rc})")
     return sorted_ids, expert_ids, int(ntp[0]), offs
+
+
+def grouped_gemm(x, qweight, scales, m_indices=None, masked_m=None, out=None, n_threads=0):
+    """Grouped GEMM: out[m] = bf16(x[m] . W[e_m]^T), FP32 accumulation; e_m from m_indices
+    (contiguous layout, -1 = no expert) or from masked_m (masked layout, x viewed as
+    [E * max_m, K]). Rows without an expert keep the contents of `out` (zeros if None)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    qw = np.ascontiguousarray(qweight, dtype=np.int32)
+    sc = np.ascontiguousarray(scales, dtype=np.uint16)
+    E, N, _ = qw.shape
+    if masked_m is not None:
+        E_, max_m, K = x.shape
+        M = E_ * max_m
+        x2 = x.reshape(M, K)
+    else:
+        M, K = x.shape
+        max_m = 0
+        x2 = x
+    res = np.zeros((M, N), dtype=np.uint16) if out is None else np.ascontiguousarray(out, dtype=np.uint16).reshape(M, N).copy()
+    mi = None if m_indices is None else np.ascontiguousarray(m_indices, dtype=np.int32)
+    mm = None if masked_m is None else np.ascontiguousarray(masked_m, dtype=np.int32)
+    rc = lib.oracle_grouped_gemm(_ptr(x2), M, K, _ptr(qw), _ptr(sc), E, N,
+                                 None if mi is None else _ptr(mi), None if mm is None else _ptr(mm),
+                                 max_m, _ptr(res), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_grouped_gemm failed ({rc})")
+    return res
 
 
 def router_topk(logits: np.ndarray, topk: int):

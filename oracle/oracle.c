@@ -23,6 +23,11 @@
  *   act      a = bf16_rne( silu(h[i]) * h[I+i] ), gate rows first, up rows second.
  *   down     y = a . W2[e]^T, FP32 accumulation.
  *   combine  out[t] = bf16_rne( sum over local slots j, ascending, of w[t,j] * y_j ).
+ *   grouped  the grouped operator on the same dequant ("Gruppierte SM90-Kernel"): rows
+ *            concatenated per expert with m_indices (-1 = padding), or a fixed row budget
+ *            per expert with masked_m valid counts; out[m] = bf16_rne( x[m] . W[e_m]^T ),
+ *            FP32 accumulation; rows without an expert are not written (consumers ignore
+ *            them, same section).
  *   router   (the step upstream of align, for the fused routing entry point) per token
  *            the topk largest logits, ties to the lower expert id, and their softmax
  *            renormalised over the chosen ones: w_r = exp(l_r - l_0) / sum_j exp(l_j - l_0)
@@ -272,5 +277,49 @@ int oracle_router_topk(const float* logits, int64_t T, int64_t G, int64_t k, int
   }
   free(taken);
   free(e);
+  return 0;
+}
+
+/* Grouped GEMM (see the header). Weights: one expert after another, qweight [E, N, K/8],
+ * scales [E, N, K/32]. Row m of x [M, K] belongs to expert e_m:
+ *   contiguous (masked_m == NULL): e_m = m_indices[m] (negative: no expert);
+ *   masked (m_indices == NULL): M = E * max_m, e_m = m / max_m when m % max_m < masked_m[e_m].
+ * out [M, N] bf16: rows with an expert get bf16_rne(sum_k x[m,k] * w[e_m][n,k]) (FP32,
+ * ascending k); other rows are left as they are. Experts are dequantised one at a time.
+ * Returns 0, or -1 for bad arguments. */
+static int64_t grouped_expert_of(int64_t m, const int32_t* m_indices, const int32_t* masked_m, int64_t max_m) {
+  if (m_indices) return m_indices[m];
+  const int64_t g = m / max_m;
+  return (m % max_m < masked_m[g]) ? g : -1;
+}
+
+int oracle_grouped_gemm(const uint16_t* x, int64_t M, int64_t K, const int32_t* qweight, const uint16_t* scales,
+                        int64_t E, int64_t N, const int32_t* m_indices, const int32_t* masked_m, int64_t max_m,
+                        uint16_t* out, int n_threads) {
+  if (M < 0 || K < 1 || N < 1 || E < 1 || (m_indices == NULL) == (masked_m == NULL)) return -1;
+  if (masked_m && (max_m < 1 || M != E * max_m)) return -1;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+  (void)n_threads;
+#endif
+  float* w = (float*)malloc((size_t)N * K * sizeof(float));
+  if (!w) return -1;
+  for (int64_t e = 0; e < E; ++e) {
+    int used = 0;
+    for (int64_t m = 0; m < M && !used; ++m) used = grouped_expert_of(m, m_indices, masked_m, max_m) == e;
+    if (!used) continue;
+    oracle_dequant(qweight + e * N * (K / 8), scales + e * N * (K / ORACLE_GROUP), N, K, w);
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t m = 0; m < M; ++m) {
+      if (grouped_expert_of(m, m_indices, masked_m, max_m) != e) continue;
+      for (int64_t n = 0; n < N; ++n) {
+        float acc = 0.0f;
+        for (int64_t k = 0; k < K; ++k) acc += oracle_bf16_to_f32(x[m * K + k]) * w[n * K + k];
+        out[m * N + n] = oracle_f32_to_bf16(acc);
+      }
+    }
+  }
+  free(w);
   return 0;
 }

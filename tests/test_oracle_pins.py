@@ -430,3 +430,139 @@ def test_router_closed_forms():
     np.testing.assert_allclose(w0, w1, rtol=2e-7)
     # weights of a row sum to one
     np.testing.assert_allclose(w0.astype(np.float64).sum(axis=1), 1.0, rtol=1e-6)
+
+
+# ------------------------------------------------------------------------------ grouped GEMM
+
+SENTINEL = np.uint16(0x7FC1)  # a NaN pattern no computed bf16 value takes
+
+
+def gcfg(mode, E, N, K, rows, max_m=0, balance="random", seed=0):
+    return inputs.GroupedConfig("t", mode, E, N, K, rows, max_m, balance, seed)
+
+
+def grouped_rows_expert(d):
+    """The expert of each flat row of x, or -1 (read off the layout's definition)."""
+    cfg = d["cfg"]
+    if cfg.mode == "contiguous":
+        return d["m_indices"].astype(np.int64)
+    r = np.arange(cfg.E * cfg.max_m)
+    e = r // cfg.max_m
+    return np.where(r % cfg.max_m < d["masked_m"][e], e, -1)
+
+
+def grouped_brute(d):
+    """Float64, weights rounded to bf16 as the method does; NaN where no expert."""
+    cfg = d["cfg"]
+    x = f32(d["x"]).reshape(-1, cfg.K)
+    ex = grouped_rows_expert(d)
+    ref = np.full((x.shape[0], cfg.N), np.nan)
+    absum = np.full_like(ref, np.nan)  # sum_k |x_k w_k|, for the rounding bound
+    for e in np.unique(ex[ex >= 0]):
+        w = dequant_f64(d["qweight"][e], d["scales"][e], rounded=True)
+        rows = ex == e
+        ref[rows] = x[rows] @ w.T
+        absum[rows] = np.abs(x[rows]) @ np.abs(w).T
+    return ref, absum
+
+
+def run_grouped_oracle(d):
+    cfg = d["cfg"]
+    M = d["x"].size // cfg.K
+    out = np.full((M, cfg.N), SENTINEL, np.uint16)
+    if cfg.mode == "contiguous":
+        return oracle.grouped_gemm(d["x"], d["qweight"], d["scales"], m_indices=d["m_indices"], out=out)
+    return oracle.grouped_gemm(d["x"], d["qweight"], d["scales"], masked_m=d["masked_m"], out=out)
+
+
+def assert_fp32_then_bf16(got_bits, ref, absum, K):
+    """A sequential FP32 sum of exact products is within (K-1) 2^-24 sum|x w| of the exact
+    sum; one bf16 rounding adds at most 2^-8 of the value."""
+    got = f32(got_bits)
+    acc = 1.01 * (K - 1) * 2.0 ** -24 * absum
+    bound = 2.0 ** -8 * (np.abs(ref) + acc) + acc
+    err = np.abs(got - ref)
+    assert np.all(err <= bound), (err.max(), np.argmax(err - bound))
+
+
+@pytest.mark.parametrize("mode,E,N,K,rows,max_m,seed", [
+    ("contiguous", 5, 256, 512, 50, 0, 1),
+    ("contiguous", 3, 384, 256, 200, 0, 2),
+    ("masked", 4, 256, 512, 40, 64, 3),
+    ("masked", 6, 128, 384, 10, 24, 4),
+])
+def test_grouped_matches_brute_force(mode, E, N, K, rows, max_m, seed):
+    d = inputs.make_grouped(gcfg(mode, E, N, K, rows, max_m, seed=seed))
+    got = run_grouped_oracle(d)
+    ref, absum = grouped_brute(d)
+    valid = grouped_rows_expert(d) >= 0
+    assert valid.any() and (~valid).any()
+    assert_fp32_then_bf16(got[valid], ref[valid], absum[valid], K)
+    assert np.all(got[~valid] == SENTINEL)  # rows without an expert are not written
+
+
+def test_grouped_masked_equals_contiguous_layout():
+    # the same valid rows in the two layouts give bit-identical results
+    d = inputs.make_grouped(gcfg("masked", 5, 256, 256, 30, 48, seed=5))
+    cfg = d["cfg"]
+    xm = d["x"].reshape(cfg.E, cfg.max_m, cfg.K)
+    got_m = run_grouped_oracle(d).reshape(cfg.E, cfg.max_m, cfg.N)
+    xs, ids = [], []
+    for e in range(cfg.E):
+        c = int(d["masked_m"][e])
+        pad = (c + 127) // 128 * 128 - c
+        xs += [xm[e, :c], np.zeros((pad, cfg.K), np.uint16)]
+        ids += [np.full(c, e, np.int32), np.full(pad, -1, np.int32)]
+    dc = {"cfg": gcfg("contiguous", cfg.E, cfg.N, cfg.K, 0), "x": np.concatenate(xs), "m_indices": np.concatenate(ids),
+          "qweight": d["qweight"], "scales": d["scales"]}
+    got_c = run_grouped_oracle(dc)
+    at = 0
+    for e in range(cfg.E):
+        c = int(d["masked_m"][e])
+        assert np.array_equal(got_c[at:at + c], got_m[e, :c])
+        at += (c + 127) // 128 * 128
+
+
+def test_grouped_relabelled_experts_give_identical_rows():
+    d = inputs.make_grouped(gcfg("contiguous", 6, 128, 256, 40, seed=6))
+    base = run_grouped_oracle(d)
+    perm = np.array([3, 5, 0, 1, 4, 2])  # expert e's weights move to slot perm[e]
+    qw, sc = np.empty_like(d["qweight"]), np.empty_like(d["scales"])
+    qw[perm], sc[perm] = d["qweight"], d["scales"]
+    mi = np.where(d["m_indices"] >= 0, perm[np.maximum(d["m_indices"], 0)], -1).astype(np.int32)
+    d2 = dict(d, qweight=qw, scales=sc, m_indices=mi)
+    assert np.array_equal(run_grouped_oracle(d2), base)
+
+
+def test_grouped_single_expert_is_dense_gemm():
+    d = inputs.make_grouped(gcfg("contiguous", 1, 256, 384, 128, balance="balanced", seed=7))
+    assert np.all(d["m_indices"] == 0)
+    w = oracle.dequant(d["qweight"][0], d["scales"][0]).astype(np.float64)
+    x = f32(d["x"])
+    ref = x @ w.T  # numpy's matmul over the oracle's own (separately pinned) dequantisation
+    assert_fp32_then_bf16(run_grouped_oracle(d), ref, np.abs(x) @ np.abs(w).T, 384)
+
+
+def test_grouped_all_equal_codes_closed_form():
+    d = inputs.make_grouped(gcfg("masked", 3, 128, 256, 20, 32, seed=8))
+    c, s_bits = 3, np.uint16(0x3CA0)  # code 3, scale 0.01953125 (exact)
+    word = np.uint32(sum(c << (4 * i) for i in range(8)))
+    d["qweight"][:] = np.array(word).view(np.int32)
+    d["scales"][:] = s_bits
+    w0 = (c - 8) * float(f32(s_bits))  # -0.09765625, a bf16 value: rounding keeps it
+    x = f32(d["x"]).reshape(-1, 256)
+    got = run_grouped_oracle(d)
+    valid = grouped_rows_expert(d) >= 0
+    ref = np.repeat((w0 * x.sum(axis=1))[:, None], 128, axis=1)  # every column the same
+    absum = np.repeat((abs(w0) * np.abs(x).sum(axis=1))[:, None], 128, axis=1)
+    assert_fp32_then_bf16(got[valid], ref[valid], absum[valid], 256)
+    assert np.all(got[valid] == got[valid][:, :1])
+
+
+def test_grouped_out_of_range_rows_are_skipped():
+    d = inputs.make_grouped(gcfg("contiguous", 4, 128, 128, 30, seed=9))
+    d["m_indices"][:7] = 4   # not an expert of this weight
+    d["m_indices"][7:9] = -3  # any negative id is padding
+    got = run_grouped_oracle(d)
+    assert np.all(got[:9] == SENTINEL)
+    assert not np.any(got[9:][d["m_indices"][9:] >= 0] == SENTINEL)

@@ -163,3 +163,78 @@ def sample_rows(topk_ids: np.ndarray, E: int, n: int = 512, seed: int = 1) -> np
         return cand.astype(np.int64)
     rng = np.random.default_rng(seed)
     return np.sort(rng.choice(cand, size=n, replace=False)).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------------
+# Grouped operator layouts ("Gruppierte SM90-Kernel"): one projection [E, N, K] applied to
+# rows already grouped by expert. Contiguous: each expert's rows consecutive, the run
+# padded to a multiple of 128 rows, m_indices = expert id or -1 for padding. Masked: a
+# fixed budget of max_m rows per expert, masked_m = valid rows. The blog measures both
+# with the same rows per expert on each side ("Messungen": grouped rows matched per expert,
+# EP8 prefill at 128 rows/expert, decode at 32 tokens/expert).
+
+@dataclasses.dataclass(frozen=True)
+class GroupedConfig:
+    name: str
+    mode: str      # 'contiguous' | 'masked'
+    E: int         # experts
+    N: int         # output columns (weight rows)
+    K: int         # reduction length
+    rows: int      # mean valid rows per expert (masked: also the expected_m hint)
+    max_m: int     # masked row budget per expert (0 for contiguous)
+    balance: str   # 'balanced': every expert has `rows`; 'random': uniform in [0, 2*rows]
+    seed: int = 0
+
+
+GROUPED_CONFIGS = {
+    # EP8 shards of Kimi-K2 (48 local experts): gate_up [4096, 7168] and down [7168, 2048]
+    "grouped_contiguous_ep8_gate_up": GroupedConfig("grouped_contiguous_ep8_gate_up", "contiguous", 48, 4096,
+                                                    7168, 128, 0, "balanced"),
+    "grouped_contiguous_ep8_down": GroupedConfig("grouped_contiguous_ep8_down", "contiguous", 48, 7168, 2048,
+                                                 128, 0, "balanced"),
+    "grouped_masked_ep8_gate_up": GroupedConfig("grouped_masked_ep8_gate_up", "masked", 48, 4096, 7168, 32, 256,
+                                                "balanced"),
+    "grouped_masked_ep8_down": GroupedConfig("grouped_masked_ep8_down", "masked", 48, 7168, 2048, 32, 256,
+                                             "balanced"),
+}
+
+
+def grouped_counts(cfg: GroupedConfig) -> np.ndarray:
+    """Valid rows per expert, int32 [E] (masked: at most max_m)."""
+    if cfg.balance == "balanced":
+        c = np.full(cfg.E, cfg.rows, dtype=np.int64)
+    elif cfg.balance == "random":
+        rng = _streams(cfg.seed)[0]
+        c = rng.integers(0, 2 * cfg.rows + 1, size=cfg.E)
+    else:
+        raise ValueError(cfg.balance)
+    if cfg.mode == "masked":
+        c = np.minimum(c, cfg.max_m)
+    return c.astype(np.int32)
+
+
+def make_grouped(cfg: GroupedConfig, weights: bool = True) -> dict:
+    """x (bf16 bits; [M, K] contiguous, [E, max_m, K] masked), m_indices int32 [M] or
+    masked_m int32 [E], and qweight int32 [E, N, K/8] / scales bf16 bits [E, N, K/32].
+    Padding rows and rows past masked_m hold random values like the rest."""
+    counts = grouped_counts(cfg)
+    _, rx, rc, rs = _streams(cfg.seed)
+    d = {"cfg": cfg, "counts": counts}
+    if cfg.mode == "contiguous":
+        runs = []
+        for e, c in enumerate(counts):
+            padded = (int(c) + 127) // 128 * 128
+            runs.append(np.concatenate([np.full(c, e, np.int32), np.full(padded - c, -1, np.int32)]))
+        m_idx = np.concatenate(runs) if runs else np.zeros(0, np.int32)
+        d["m_indices"] = m_idx.astype(np.int32)
+        shape = (m_idx.size, cfg.K)
+    elif cfg.mode == "masked":
+        d["masked_m"] = counts
+        shape = (cfg.E, cfg.max_m, cfg.K)
+    else:
+        raise ValueError(cfg.mode)
+    d["x"] = _f32_to_bf16_bits_trunc(rx.standard_normal(shape, dtype=np.float32))
+    if weights:
+        d["qweight"] = _codes(rc, cfg.E, cfg.N, cfg.K)
+        d["scales"] = _scales(rs, cfg.E, cfg.N, cfg.K)
+    return d
