@@ -2,7 +2,9 @@
 """Benchmark of the B200 W4A16 mixture-of-experts layer.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl chord|reference]
-                    [--workload ep8_decode|ep8_prefill|tp8_decode|tp8_prefill|skew|tiny]
+                    [--workload ep8_decode|ep8_prefill|tp8_decode|tp8_prefill|skew|tiny
+                                |grouped_contiguous_ep8_gate_up|grouped_contiguous_ep8_down
+                                |grouped_masked_ep8_gate_up|grouped_masked_ep8_down]
 
 One step = one layer call through the C ABI: routing sort (chord_moe_align) then
 chord_moe_forward (gate_up GEMM + SiLU*up, down GEMM + top-k weight, combine), on a
@@ -14,6 +16,10 @@ so no flush is needed between steps.
 Prints one JSON line (rank 0). `value` is microseconds per layer call for the whole job:
 the max over ranks of the timed region divided by (steps x ranks), since each rank runs
 an independent replica (the layer does not shard across GPUs here).
+
+The grouped_* workloads time the grouped operators instead (one step = one
+chord_grouped_contiguous / chord_grouped_masked call: routing pass + GEMM) on an EP8 shard
+(48 experts) at the rows per expert the blog's grouped table uses.
 
 --impl reference times the CPU oracle (test infrastructure) on the same workload on
 the host cores: rank 0 only, other ranks exit without work.
@@ -375,6 +381,192 @@ def time_router(chord, cfg, rcfg, dev, calls=20, replays=10):
     return a.elapsed_time(b) * 1000.0 / (calls * replays)
 
 
+# ------------------------------------------------------------------------------ grouped operators
+
+GROUPED_METRIC = "W4A16 grouped GEMM µs/call; eff. HBM GB/s (masked decode) or TFLOPS (contiguous prefill)"
+
+
+def describe_grouped(cfg) -> str:
+    lay = (f"masked, max_m={cfg.max_m}, masked_m={cfg.rows} ({cfg.balance})" if cfg.mode == "masked"
+           else f"contiguous, {cfg.rows} rows/expert ({cfg.balance}), runs padded to 128")
+    return (f"{cfg.name}: E={cfg.E} N={cfg.N} K={cfg.K}, {lay}, int4 group-32 bf16 scales")
+
+
+def grouped_work(cfg, counts):
+    valid = int(counts.sum())
+    active = int((counts > 0).sum())
+    w_bytes = active * (cfg.N * cfg.K // 2 + cfg.N * (cfg.K // 32) * 2)
+    return {"valid_rows": valid, "active_experts": active,
+            "bytes": w_bytes + valid * cfg.K * 2 + valid * cfg.N * 2,
+            "flops": 2 * valid * cfg.N * cfg.K}
+
+
+def run_grouped(args, rank, world, local_rank):
+    """One step = one grouped operator call (routing pass + GEMM) through the C ABI."""
+    import torch
+    from w4a16_int4_mixture_align_b200 import chord
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = inputs.GROUPED_CONFIGS[args.workload]
+    d = inputs.make_grouped(inputs.GroupedConfig(**{**cfg.__dict__, "seed": cfg.seed + rank}))
+    work = grouped_work(cfg, d["counts"])
+    w = chord.pack_w4a16_grouped(d["qweight"], d["scales"].view(np.int16), cfg.mode, device=dev)
+    del d["qweight"], d["scales"]
+    x_np = d["x"]
+    x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    M = x_np.size // cfg.K
+    out = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+    route_np = d["m_indices"] if cfg.mode == "contiguous" else d["masked_m"]
+    route = torch.from_numpy(route_np).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    flags = {"auto": 0, "stream": chord.CHORD_FLAG_FORCE_STREAM, "tensor": chord.CHORD_FLAG_FORCE_TENSOR}[args.schedule]
+    expected_m = args.expected_m or cfg.rows
+
+    def call(xx, rr, oo):
+        if cfg.mode == "contiguous":
+            chord.contiguous(xx, w, rr, out=oo, flags=flags)
+        else:
+            chord.masked(xx, w, rr, expected_m, out=oo, flags=flags)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        call(x, route, out)
+    torch.cuda.synchronize()
+    assert w.check_status() == 0
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    launches0 = chord.chord_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for k in range(K):
+            ev[k][0].record(stream)
+            chord.chord_set_timing_events([ev[k][1], ev[k][2], ev[k][2], ev[k][2]])
+            call(x, route, out)
+            chord.chord_set_timing_events(None)
+    launches = chord.chord_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    graph.replay()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    elapsed_ms = start.elapsed_time(stop)
+    assert w.check_status() == 0
+    del graph
+    seg = np.array([[ev[k][0].elapsed_time(ev[k][1]), ev[k][1].elapsed_time(ev[k][2])] for k in range(K)])
+    seg_ms = seg.mean(axis=0)  # routing pass, GEMM
+
+    # end to end: activations and routing from pinned host memory, the result back
+    x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
+    r_h = torch.from_numpy(route_np).pin_memory()
+    out_h = torch.empty((M, cfg.N), dtype=torch.int16).pin_memory()
+    xd, rd = torch.empty_like(x), torch.empty_like(route)
+
+    def e2e_step():
+        xd.view(torch.int16).copy_(x_h, non_blocking=True)
+        rd.copy_(r_h, non_blocking=True)
+        call(xd, rd, out)
+        out_h.copy_(out.view(torch.int16), non_blocking=True)
+
+    for _ in range(W):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler.stop()
+    e2e_ms = s2.elapsed_time(e2)
+    stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
+    elapsed_ms, e2e_ms, seg_ms = stats[0], stats[1], np.array(stats[2:])
+    if rank != 0:
+        return None
+
+    hbm, tf_burst, tf_sust, pk_kind = peaks()
+    gemm_us = seg_ms[1] * 1000.0
+    # the library's default schedule: expected rows per expert (masked: the expected_m hint;
+    # contiguous: padded rows / E) above 16 go to the tensor cores
+    expected = expected_m if cfg.mode == "masked" else -(-M // cfg.E)
+    tensor = args.schedule == "tensor" or (args.schedule == "auto" and expected > 16)
+    unit = ((32 if expected <= 32 else 64 if expected <= 64 else 128 if expected <= 128 else 256) if tensor
+            else (8 if expected <= 8 else (16 if expected <= 16 else 32)))
+    if tensor:
+        achieved = work["flops"] / (gemm_us * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": "tc_gemm (plain epilogue)", "achieved": round(achieved, 1),
+                    "peak": tf_sust, "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
+                    "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long run of calls)",
+                    "peak_burst": tf_burst, "frac_of_burst": round(achieved / tf_burst, 4),
+                    "traffic": recorded_traffic("tc_gemm_plain", args.workload),
+                    "algorithmic_flops_per_launch": work["flops"]}
+    else:
+        achieved = work["bytes"] / (gemm_us * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "kernel": "stream_gemm (plain epilogue)", "achieved": round(achieved, 1),
+                    "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": f"{pk_kind} hbm_gbs",
+                    "traffic": recorded_traffic("stream_gemm_plain", args.workload),
+                    "algorithmic_bytes_per_launch": work["bytes"]}
+    return {
+        "metric": GROUPED_METRIC, "value": round(job_us_per_call(elapsed_ms, K, world), 3), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(elapsed_ms / K, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe_grouped(cfg), "schedule": "tensor-core" if tensor else "weight-streaming",
+                   "unit_rows": unit, "expected_m": expected_m if cfg.mode == "masked" else None,
+                   "valid_rows": work["valid_rows"], "active_experts": work["active_experts"],
+                   "l2": "no flush: weights %.2f GB > 126 MB L2" % (work["bytes"] / 1e9),
+                   "parallelism": f"replicas x{world}"},
+        "kernels_us": {"routing": round(seg_ms[0] * 1000, 2), "gemm": round(gemm_us, 2)},
+        "roofline": roofline,
+        "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
+                "h2d_bytes_per_step": x_h.numel() * 2 + r_h.numel() * 4, "d2h_bytes_per_step": out_h.numel() * 2},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+
+
+def grouped_cpu_baseline(cfg, n_experts=2, d=None):
+    """The oracle's grouped GEMM on a bounded sample: every valid row of n_experts experts
+    (seeded choice among the active ones), scaled to the full call by active experts."""
+    import oracle
+    oracle.build()
+    d = inputs.make_grouped(cfg) if d is None else d
+    if cfg.mode == "contiguous":
+        ex = d["m_indices"].astype(np.int64)
+    else:
+        r = np.arange(cfg.E * cfg.max_m)
+        ex = np.where(r % cfg.max_m < d["masked_m"][r // cfg.max_m], r // cfg.max_m, -1)
+    active = np.unique(ex[ex >= 0])
+    pick = np.random.default_rng(0).choice(active, min(n_experts, active.size), replace=False)
+    rows = np.nonzero(np.isin(ex, pick))[0]
+    threads = os.cpu_count() or 1
+    t0 = time.time()
+    oracle.grouped_gemm(d["x"].reshape(-1, cfg.K)[rows], d["qweight"], d["scales"],
+                        m_indices=ex[rows].astype(np.int32), n_threads=threads)
+    el = time.time() - t0
+    us = el * 1e6 * active.size / pick.size
+    return {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"all {rows.size} valid rows of {pick.size} of {active.size} active experts "
+                      f"(seeded), scaled by active experts"}
+
+
 def max_over_ranks(vals, world, device=None):
     """Element-wise max of `vals` over all ranks (one all-reduce; identity for world 1)."""
     import torch
@@ -429,6 +621,8 @@ def run_reference(args, rank, world):
         return None
     import oracle
     oracle.build()
+    if args.workload in inputs.GROUPED_CONFIGS:
+        return run_reference_grouped(args, world)
     cfg = inputs.CONFIGS[args.workload]
     d = inputs.make_inputs(cfg)
     threads = os.cpu_count() or 1
@@ -450,6 +644,26 @@ def run_reference(args, rank, world):
     }
 
 
+def run_reference_grouped(args, world):
+    """Each step: the oracle's grouped GEMM on a 64-row seeded sample of the workload,
+    scaled to the full call by valid rows."""
+    cfg = inputs.GROUPED_CONFIGS[args.workload]
+    d = inputs.make_grouped(cfg)
+    for _ in range(args.warmup):
+        grouped_cpu_baseline(cfg, d=d)
+    vals = [grouped_cpu_baseline(cfg, d=d) for _ in range(args.steps)]
+    us = statistics.mean(v["value"] for v in vals)
+    base = dict(vals[0], value=round(us, 1))
+    return {
+        "impl": "reference", "metric": GROUPED_METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": describe_grouped(cfg), "parallelism": "rank 0 only"},
+        "cpu_baseline": base,
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 # ------------------------------------------------------------------------------ main
 
 def main():
@@ -458,11 +672,16 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["chord", "reference"], default="chord")
-    ap.add_argument("--workload", choices=list(inputs.CONFIGS), default="ep8_decode")
+    ap.add_argument("--workload", choices=list(inputs.CONFIGS) + sorted(inputs.GROUPED_CONFIGS),
+                    default="ep8_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", choices=["auto", "stream", "tensor"], default="auto",
+                    help="grouped workloads: force the GEMM schedule")
+    ap.add_argument("--expected-m", type=int, default=None,
+                    help="grouped masked workloads: the expected_m hint (default: the rows per expert)")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = 3 if args.impl == "reference" else DEFAULT_STEPS[args.workload]
+        args.steps = 3 if args.impl == "reference" else DEFAULT_STEPS.get(args.workload, 200)
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -482,10 +701,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
 
-    line = run_chord(args, rank, world, local_rank)
+    grouped = args.workload in inputs.GROUPED_CONFIGS
+    line = (run_grouped if grouped else run_chord)(args, rank, world, local_rank)
     if line is not None:
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(inputs.CONFIGS[args.workload])
+            line["cpu_baseline"] = (grouped_cpu_baseline(inputs.GROUPED_CONFIGS[args.workload]) if grouped
+                                    else cpu_baseline(inputs.CONFIGS[args.workload]))
         else:
             line["cpu_baseline"] = None
     if world > 1:

@@ -68,6 +68,8 @@ typedef enum {
 /* Weight roles for chord_repack_weights. */
 #define CHORD_ROLE_GATE_UP 1 /* W13 [E, 2I, H]: rows [0,I) gate, rows [I,2I) up */
 #define CHORD_ROLE_DOWN    2 /* W2  [E, H, I] */
+#define CHORD_ROLE_GROUPED_CONTIGUOUS 3 /* W [E, N, K] for chord_grouped_contiguous */
+#define CHORD_ROLE_GROUPED_MASKED     4 /* W [E, N, K] for chord_grouped_masked */
 
 /* Flags for chord_moe_forward. */
 #define CHORD_FLAG_VALIDATE_ROUTING 0x1 /* check routing tensors on the device first */
@@ -225,13 +227,61 @@ CHORD_API chord_status_t chord_moe_check_status(void* workspace, chord_stream_t 
                                       uint32_t* device_status);
 
 /* ------------------------------------------------------------------------------------
+ * Grouped operators ("Gruppierte SM90-Kernel": the second operator family, with its own
+ * routing layouts; "Gruppierte Operatoreintrittspunkte": contiguous for prefill, masked
+ * for decode). Each computes, for every row m of x that belongs to an expert e_m,
+ *     out[m, n] = bf16_rne( sum_k x[m, k] * w[e_m][n, k] ),  w = bf16((q - 8) * s),
+ * with FP32 accumulation (the dequantisation of the indexed path). Rows that belong to
+ * no expert are not written: the caller ignores them.
+ *
+ * chord_grouped_contiguous: rows concatenated by expert, each expert's run padded to a
+ *   multiple of 128 rows ("Kontiguoeser Prefill").
+ *   x         device bf16 [M, K], 16-byte aligned
+ *   m_indices device int32 [M], 16-byte aligned: the expert of each row in [0, E), or
+ *             a negative id for padding.
+ *             Every aligned 128-row block (rows 128b .. 128b+127) must hold rows of at
+ *             most one expert; a block that mixes experts or names an id >= E is not
+ *             computed and sets CHORD_DEV_ROUTING_INVALID in the workspace status.
+ *   out       device bf16 [M, N], 16-byte aligned
+ * chord_grouped_masked: a fixed row budget per expert ("Maskierter Decode").
+ *   x         device bf16 [E, max_m, K] (= [E * max_m, K]), 16-byte aligned
+ *   masked_m  device int32 [E]: the valid rows of each expert; rows m with
+ *             m % max_m >= masked_m[m / max_m] are not written. Counts outside
+ *             [0, max_m] are clamped and set CHORD_DEV_ROUTING_INVALID.
+ *   expected_m host hint (> 0), the rows per expert the caller expects; it only picks
+ *             the schedule and never changes results.
+ *   out       device bf16 [E * max_m, N] (flat even when x is 3-D)
+ * Both: w is a blob from chord_repack_weights with the matching role
+ *   (CHORD_ROLE_GROUPED_CONTIGUOUS / CHORD_ROLE_GROUPED_MASKED) and shape [E, N, K]; a
+ *   blob of another role or shape fails with CHORD_ERR_LAYOUT_MISMATCH (prepared in this
+ *   process) or sets CHORD_DEV_BLOB_MISMATCH (foreign blob: the kernel reads its
+ *   header). N % 128 == 0, K % 128 == 0, 1 <= E <= 1024.
+ *   workspace: device, >= chord_grouped_workspace_bytes(rows, E) bytes, rows = M or
+ *   E * max_m, 256-byte aligned; its first 256 bytes hold the status word as for
+ *   chord_moe_forward (zero once; read with chord_moe_check_status).
+ *   flags: CHORD_FLAG_FORCE_STREAM / CHORD_FLAG_FORCE_TENSOR pick the schedule; by
+ *   default expected rows per expert (M / E, or expected_m) <= 16 streams the weights.
+ *   Two kernels run on `stream`: a routing pass over m_indices / masked_m, then the GEMM;
+ *   nothing is read back to the host, so both calls can be captured in a CUDA graph.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API size_t chord_grouped_workspace_bytes(int64_t rows, int E);
+CHORD_API chord_status_t chord_grouped_contiguous(const uint16_t* x, int64_t M, int K, const int32_t* m_indices,
+                                                  const void* w, int E, int N, uint16_t* out, void* workspace,
+                                                  size_t workspace_bytes, int flags, chord_stream_t stream);
+CHORD_API chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t max_m, int K,
+                                              const int32_t* masked_m, int64_t expected_m, const void* w, int N,
+                                              uint16_t* out, void* workspace, size_t workspace_bytes, int flags,
+                                              chord_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used by the benchmark).
  *
  * chord_set_timing_events: while set (n == 4), every chord_moe_forward made on the
  * calling thread records the caller-owned cudaEvent_t handles events[0..3] on its
  * stream: [0] right before the gate_up GEMM kernel (after routing validation and, on
  * the tensor-core schedule, the row permutation), [1] between the gate_up and down GEMM
- * kernels, [2] after the down GEMM, [3] after the combine. Records use cudaEventRecordExternal,
+ * kernels, [2] after the down GEMM, [3] after the combine. The grouped operators record
+ * [0] right before their GEMM kernel and [1] after it. Records use cudaEventRecordExternal,
  * so a forward captured into a CUDA graph records them when the graph is replayed. n == 0 clears the hook. The handles must stay
  * valid while set. Returns CHORD_ERR_INVALID_ARG for other n or null handles.
  *

@@ -61,7 +61,7 @@ def tiny():
     return inputs.make_inputs(inputs.CONFIGS["tiny"])
 
 
-@pytest.mark.parametrize("block_m", [1, 8, 16, 32, 64, 256])
+@pytest.mark.parametrize("block_m", [1, 8, 16, 32, 64, 144, 240, 256])
 @pytest.mark.parametrize("path", ["stream", "tensor"])
 def test_tiny_full_output(chord, tiny, block_m, path):
     flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR

@@ -28,6 +28,8 @@ CHORD_DEV_TIMEOUT = 0x4
 
 CHORD_ROLE_GATE_UP = 1
 CHORD_ROLE_DOWN = 2
+CHORD_ROLE_GROUPED_CONTIGUOUS = 3
+CHORD_ROLE_GROUPED_MASKED = 4
 
 CHORD_FLAG_VALIDATE_ROUTING = 0x1
 CHORD_FLAG_FORCE_STREAM = 0x2
@@ -55,6 +57,9 @@ SIGNATURES = {
     "chord_moe_check_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "chord_moe_align_noalloc": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "chord_router_topk_align": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "chord_grouped_workspace_bytes": (_SZ, [_I64, _I]),
+    "chord_grouped_contiguous": (_I, [_P, _I64, _I, _P, _P, _I, _I, _P, _P, _SZ, _I, _P]),
+    "chord_grouped_masked": (_I, [_P, _I, _I64, _I, _P, _I64, _P, _I, _P, _P, _SZ, _I, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
 }
@@ -196,6 +201,26 @@ def chord_moe_forward(hidden, topk_ids, topk_weights, sorted_ids, expert_ids, nu
            "chord_moe_forward")
 
 
+def chord_grouped_workspace_bytes(rows, E) -> int:
+    return int(lib().chord_grouped_workspace_bytes(rows, E))
+
+
+def chord_grouped_contiguous(x, m_indices, w, E, N, out, workspace, flags=0, stream=None):
+    M, K = x.shape
+    _check(lib().chord_grouped_contiguous(_ptr(x), M, K, _ptr(m_indices), _ptr(w), E, N, _ptr(out),
+                                          _ptr(workspace), _nbytes(workspace), flags, _stream(stream)),
+           "chord_grouped_contiguous")
+
+
+def chord_grouped_masked(x, masked_m, expected_m, w, N, out, workspace, flags=0, stream=None):
+    E = masked_m.shape[0]
+    K = x.shape[-1]
+    max_m = x.shape[1] if x.dim() == 3 else x.shape[0] // E  # [E, max_m, K] or [E * max_m, K]
+    _check(lib().chord_grouped_masked(_ptr(x), E, max_m, K, _ptr(masked_m), int(expected_m), _ptr(w), N,
+                                      _ptr(out), _ptr(workspace), _nbytes(workspace), flags, _stream(stream)),
+           "chord_grouped_masked")
+
+
 def chord_moe_check_status(workspace, stream=None) -> int:
     v = ctypes.c_uint32(0)
     st = lib().chord_moe_check_status(_ptr(workspace), _stream(stream), ctypes.byref(v))
@@ -287,3 +312,58 @@ class ChordMoE:
 
     def check_status(self) -> int:
         return chord_moe_check_status(self.workspace)
+
+
+class GroupedWeight:
+    """A weight prepared for one grouped operator ("Gruppierte Operatoreintrittspunkte":
+    the mode is part of the prepared weight and checked when the operator runs).
+
+    qweight int32 [E, N, K/8] (eight codes per word, low nibble first), scales bf16 bits
+    [E, N, K/32]; mode "contiguous" or "masked". Keeps a workspace for its calls.
+    """
+
+    def __init__(self, qweight, scales, mode, device="cuda"):
+        roles = {"contiguous": CHORD_ROLE_GROUPED_CONTIGUOUS, "masked": CHORD_ROLE_GROUPED_MASKED}
+        if mode not in roles:
+            raise ValueError(f"mode must be 'contiguous' or 'masked', not {mode!r}")
+        self.mode, self.role = mode, roles[mode]
+        self.E, self.N, K8 = qweight.shape
+        self.K = K8 * 8
+        self.device = torch.device(device)
+        self.blob = _alloc_bytes(chord_repacked_bytes(self.E, self.N, self.K), self.device)
+        dev = lambda a: torch.as_tensor(a).to(self.device).contiguous()  # noqa: E731
+        chord_repack_weights(dev(qweight), dev(scales), self.role, self.blob)
+        self.workspace = None
+
+    def _workspace(self, rows):
+        need = chord_grouped_workspace_bytes(rows, self.E)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=self.device)
+        return self.workspace
+
+    def check_status(self) -> int:
+        return 0 if self.workspace is None else chord_moe_check_status(self.workspace)
+
+
+def pack_w4a16_grouped(qweight, scales, mode, device="cuda") -> GroupedWeight:
+    return GroupedWeight(qweight, scales, mode, device)
+
+
+def contiguous(a2, weight: GroupedWeight, m_indices, out=None, flags=0):
+    """out [M, N] bf16 for rows grouped by expert (m_indices: expert or -1 per row)."""
+    M = a2.shape[0]
+    if out is None:
+        out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=a2.device)
+    chord_grouped_contiguous(a2, m_indices, weight.blob, weight.E, weight.N, out, weight._workspace(M), flags)
+    return out
+
+
+def masked(a3, weight: GroupedWeight, masked_m, expected_m, out=None, flags=0):
+    """out [E * max_m, N] bf16 (flat); rows past masked_m[e] in each expert are not written.
+    a3 is [E, max_m, K] or [E * max_m, K]."""
+    E = weight.E
+    max_m = a3.shape[1] if a3.dim() == 3 else a3.shape[0] // E
+    if out is None:
+        out = torch.empty((E * max_m, weight.N), dtype=torch.bfloat16, device=a3.device)
+    chord_grouped_masked(a3, masked_m, expected_m, weight.blob, weight.N, out, weight._workspace(E * max_m), flags)
+    return out

@@ -184,7 +184,7 @@ chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scal
   g_detail[0] = 0;
   if (group_size != kGroup)
     return fail(CHORD_ERR_UNSUPPORTED, "group_size=%d; only group-32 scales are supported", group_size);
-  if (role != CHORD_ROLE_GATE_UP && role != CHORD_ROLE_DOWN)
+  if (role < CHORD_ROLE_GATE_UP || role > CHORD_ROLE_GROUPED_MASKED)
     return fail(CHORD_ERR_INVALID_ARG, "role=%d", role);
   if (E < 1 || N < 1 || K < 1) return fail(CHORD_ERR_INVALID_ARG, "E=%d N=%d K=%d", E, N, K);
   if (N % kTileN || K % kTileK)
@@ -344,6 +344,112 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   if (timing && (err = record_timing_event(g_timing[3], stream)) != cudaSuccess)
     return cuda_fail(err, "timing event");
   return CHORD_OK;
+}
+
+size_t chord_grouped_workspace_bytes(int64_t rows, int E) {
+  if (rows < 0 || E < 1) return 0;
+  return size_t(grouped_workspace(rows, E).total);
+}
+
+namespace {
+
+// Shared part of the two grouped entry points: checks, the routing pass, the GEMM.
+chord_status_t grouped_gemm(const uint16_t* x, int64_t rows, int K, const int32_t* m_indices,
+                            const int32_t* masked_m, int64_t max_m, int64_t expected, const void* w, int E, int N,
+                            uint16_t* out, void* workspace, size_t workspace_bytes, int flags, int role,
+                            cudaStream_t stream) {
+  if (E < 1 || E > 1024) return fail(CHORD_ERR_UNSUPPORTED, "E=%d outside [1, 1024]", E);
+  if (K < kTileK || K % kTileK || N < kTileN || N % kTileN)
+    return fail(CHORD_ERR_UNSUPPORTED, "N=%d and K=%d must be positive multiples of 128", N, K);
+  if (rows < 0 || rows >= (int64_t(1) << 31) - 256)
+    return fail(rows < 0 ? CHORD_ERR_INVALID_ARG : CHORD_ERR_UNSUPPORTED, "rows=%lld", (long long)rows);
+  if ((flags & CHORD_FLAG_FORCE_STREAM) && (flags & CHORD_FLAG_FORCE_TENSOR))
+    return fail(CHORD_ERR_INVALID_ARG, "FORCE_STREAM and FORCE_TENSOR are exclusive");
+  if (!w || !workspace) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if (rows > 0 && (!x || !out || (!m_indices && !masked_m)))
+    return fail(CHORD_ERR_INVALID_ARG, "null activation or routing pointer");
+  if (!aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(m_indices)) & 15)
+    return fail(CHORD_ERR_INVALID_ARG, "x, out and m_indices must be 16-byte aligned");
+  const GroupedWorkspace ws = grouped_workspace(rows, E);
+  if (workspace_bytes < size_t(ws.total))
+    return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "grouped workspace needs %llu bytes, got %zu",
+                (unsigned long long)ws.total, workspace_bytes);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_blobs.find(w);
+    if (it != g_blobs.end()) {  // foreign blobs: the kernels check their header
+      const BlobInfo& b = it->second;
+      if (b.role != role || b.E != E || b.N != N || b.K != K)
+        return fail(CHORD_ERR_LAYOUT_MISMATCH,
+                    "weight blob is role %d [E=%d N=%d K=%d], call needs role %d [E=%d N=%d K=%d]", b.role, b.E,
+                    b.N, b.K, role, E, N, K);
+    }
+  }
+  chord_status_t st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if (rows == 0) return CHORD_OK;
+
+  // schedule: few rows per expert stream the weights (mma.sync over units of 8, 16 or 32
+  // rows, one token chunk each); more go to the tensor cores, with units of 32 to 256 rows
+  // sized to the expected rows (a smaller unit leaves room for deeper operand rings)
+  const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) || (!(flags & CHORD_FLAG_FORCE_STREAM) && expected > 16);
+  const int bm = tensor ? (expected <= 32 ? 32 : expected <= 64 ? 64 : expected <= 128 ? 128 : 256)
+                        : (expected <= 8 ? 8 : (expected <= 16 ? 16 : 32));
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  GroupedArgs g{};
+  g.x = x;
+  g.rows = rows;
+  g.K = K;
+  g.N = N;
+  g.E = E;
+  g.role = role;
+  g.w = static_cast<const uint8_t*>(w);
+  g.out = out;
+  g.expert_ids = reinterpret_cast<int32_t*>(wsb + ws.expert_ids_offset);
+  g.block_row0 = reinterpret_cast<int32_t*>(wsb + ws.block_row0_offset);
+  g.sorted_ids = reinterpret_cast<int32_t*>(wsb + ws.sorted_ids_offset);
+  g.ntp = reinterpret_cast<int32_t*>(wsb + ws.ntp_offset);
+  g.bm = bm;
+  g.cap = ws.max_positions;
+  g.status = reinterpret_cast<uint32_t*>(wsb);
+  g.num_sms = dev.num_sms;
+  cudaError_t err = launch_grouped_route(m_indices, rows, masked_m, E, max_m, bm,
+                                         const_cast<int32_t*>(g.expert_ids), const_cast<int32_t*>(g.block_row0),
+                                         const_cast<int32_t*>(g.sorted_ids), const_cast<int32_t*>(g.ntp), g.status,
+                                         stream);
+  if (err != cudaSuccess) return cuda_fail(err, "grouped routing launch");
+  const bool timing = g_timing_on;
+  if (timing && (err = record_timing_event(g_timing[0], stream)) != cudaSuccess) return cuda_fail(err, "timing event");
+  err = tensor ? launch_tc_grouped(g, stream) : launch_stream_grouped(g, stream);
+  if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");
+  if (timing && (err = record_timing_event(g_timing[1], stream)) != cudaSuccess) return cuda_fail(err, "timing event");
+  return CHORD_OK;
+}
+
+}  // namespace
+
+chord_status_t chord_grouped_contiguous(const uint16_t* x, int64_t M, int K, const int32_t* m_indices,
+                                        const void* w, int E, int N, uint16_t* out, void* workspace,
+                                        size_t workspace_bytes, int flags, chord_stream_t stream) {
+  g_detail[0] = 0;
+  if (M < 0) return fail(CHORD_ERR_INVALID_ARG, "M=%lld", (long long)M);
+  const int64_t expected = E > 0 ? (M + E - 1) / E : 0;
+  return grouped_gemm(x, M, K, m_indices, nullptr, 0, expected, w, E, N, out, workspace, workspace_bytes, flags,
+                      CHORD_ROLE_GROUPED_CONTIGUOUS, reinterpret_cast<cudaStream_t>(stream));
+}
+
+chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t max_m, int K, const int32_t* masked_m,
+                                    int64_t expected_m, const void* w, int N, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int flags, chord_stream_t stream) {
+  g_detail[0] = 0;
+  if (max_m < 1 || expected_m < 1)
+    return fail(CHORD_ERR_INVALID_ARG, "max_m=%lld expected_m=%lld", (long long)max_m, (long long)expected_m);
+  if (E < 1 || E > 1024) return fail(CHORD_ERR_UNSUPPORTED, "E=%d outside [1, 1024]", E);
+  if (!masked_m) return fail(CHORD_ERR_INVALID_ARG, "null masked_m");
+  return grouped_gemm(x, int64_t(E) * max_m, K, nullptr, masked_m, max_m, expected_m, w, E, N, out, workspace,
+                      workspace_bytes, flags, CHORD_ROLE_GROUPED_MASKED, reinterpret_cast<cudaStream_t>(stream));
 }
 
 chord_status_t chord_set_timing_events(void* const* events, int n) {

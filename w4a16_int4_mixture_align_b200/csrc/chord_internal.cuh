@@ -327,6 +327,37 @@ struct ForwardArgs {
   int num_sms;
 };
 
+// Grouped operators: workspace layout for `rows` rows of x (M, or E * max_m) and E
+// experts, for any unit size bm in {8, 16, 32, 64, 128, 256}.
+struct GroupedWorkspace {
+  int64_t max_units, max_positions, ntp_offset, expert_ids_offset, block_row0_offset, sorted_ids_offset, total;
+};
+GroupedWorkspace grouped_workspace(int64_t rows, int E);
+// The routing pass: m_indices (contiguous, 16-byte aligned) or masked_m (masked) -> units
+// of bm rows, bm in {8, 16, 32, 64, 128, 256}.
+cudaError_t launch_grouped_route(const int32_t* m_indices, int64_t M, const int32_t* masked_m, int E,
+                                 int64_t max_m, int bm, int32_t* expert_ids, int32_t* block_row0,
+                                 int32_t* sorted_ids, int32_t* ntp, uint32_t* status, cudaStream_t stream);
+
+struct GroupedArgs {
+  const uint16_t* x;        // [rows, K]
+  int64_t rows;
+  int K, N, E, role;
+  const uint8_t* w;         // blob
+  uint16_t* out;            // [rows, N]
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* block_row0;
+  const int32_t* ntp;
+  int bm;                   // positions per unit
+  int64_t cap;              // sorted_ids capacity
+  uint32_t* status;
+  int num_sms;
+};
+// The GEMM of the grouped operators: out[row] = x[row] . W[e]^T for every valid row.
+cudaError_t launch_tc_grouped(const GroupedArgs& g, cudaStream_t stream);
+cudaError_t launch_stream_grouped(const GroupedArgs& g, cudaStream_t stream);  // token chunk = g.bm
+
 // Adds n to the process-wide kernel launch counter (chord_launch_count).
 void count_launches(int n);
 

@@ -35,7 +35,9 @@ constexpr int kThreads = 32 * (1 + kConsumerWarps);
 constexpr int kDescRing = 32;
 constexpr int kMaxTC = 32;
 
-enum Epi { kGateUp = 0, kDown = 1 };
+// kGateUp: SiLU(gate) * up into a; kDown: fp32 y by flat slot; kPlain: bf16 out[row, n]
+// with the activation row taken from sorted_ids (grouped operators).
+enum Epi { kGateUp = 0, kDown = 1, kPlain = 2 };
 
 struct StreamParams {
   const uint8_t* tiles;     // blob tile region
@@ -51,6 +53,7 @@ struct StreamParams {
   int64_t n_slots;          // T * topk
   int topk;
   int64_t cap;
+  uint16_t* out;            // kPlain output [rows, N]
   uint16_t* a_out;          // gate_up output [cap, I]
   float* y_out;             // down output [T*topk, H]
   const float* topk_weights;
@@ -318,7 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 #pragma unroll
     for (int n8 = 0; n8 < NT8; ++n8) {
       const int f = d.f[n8 * 8 + g];
-      const int64_t row = f < 0 ? 0 : ((EPI == kGateUp) ? int64_t(f / p.topk) : int64_t(d.pos0 + n8 * 8 + g));
+      const int64_t row = f < 0 ? 0
+                          : (EPI == kGateUp ? int64_t(f / p.topk)
+                                            : (EPI == kPlain ? int64_t(f) : int64_t(d.pos0 + n8 * 8 + g)));
       xrow0[n8] = p.act + row * p.act_ld;
     }
     // independent accumulator chains per 8-token tile so consecutive MMAs overlap
@@ -376,6 +381,20 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
           if (d.f[col] >= 0) {
             const float v = silu_mul(accs[n8][q], accs[n8][2 + q]);
             p.a_out[int64_t(d.pos0 + col) * p.I + i_col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          }
+        }
+      }
+    } else if (EPI == kPlain) {
+      const int n0 = d.nt * kTileN + rb * 16 + g;
+#pragma unroll
+      for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int f = d.f[n8 * 8 + 2 * t + q];
+          if (f >= 0) {
+            uint16_t* orow = p.out + int64_t(f) * p.N;
+            orow[n0] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][q]));
+            orow[n0 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][2 + q]));
           }
         }
       }
@@ -464,6 +483,31 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
   p.act = a.a;
   p.act_ld = a.I;
   return launch_tc<kDown>(p, tc, grid, stream);
+}
+
+cudaError_t launch_stream_grouped(const GroupedArgs& g, cudaStream_t stream) {
+  // one token chunk per routing unit
+  if (g.bm != 8 && g.bm != 16 && g.bm != 32) return cudaErrorInvalidValue;
+  const int tc = g.bm;
+  StreamParams p{};
+  p.ntp = g.ntp;
+  p.sorted_ids = g.sorted_ids;
+  p.expert_ids = g.expert_ids;
+  p.block_m = g.bm;
+  p.n_slots = g.rows;  // sorted_ids holds x rows
+  p.topk = 1;
+  p.cap = g.cap;
+  p.out = g.out;
+  p.E = g.E;
+  p.status = g.status;
+  p.blob = g.w;
+  p.tiles = g.w + blob_tiles_offset();
+  p.N = g.N;
+  p.K = g.K;
+  p.role = g.role;
+  p.act = g.x;
+  p.act_ld = g.K;
+  return launch_tc<kPlain>(p, tc, g.num_sms, stream);
 }
 
 }  // namespace chord

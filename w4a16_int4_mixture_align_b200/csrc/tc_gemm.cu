@@ -71,7 +71,7 @@ namespace chord {
 namespace {
 
 constexpr int kRawTiles = 2;      // 128-wide K tiles per raw stage (one bulk copy)
-constexpr int kRawStages = 3;
+constexpr int kMaxRawStages = 8;  // upper bound of the raw weight ring (runtime sized, >= 3)
 constexpr int kMaxStages = 8;     // upper bound of the A and B rings (runtime sized)
 constexpr int kMaxN = 256;
 constexpr int kDescRingTC = 8;
@@ -94,7 +94,7 @@ struct TcDesc {
 // fixed part (from the 1024-aligned base): descriptors, barriers, TMEM slot; then rings
 constexpr int kOffDesc = 0;
 constexpr int kOffBar = kOffDesc + kDescRingTC * int(sizeof(TcDesc));
-constexpr int kNumBars = 2 * kRawStages + 4 * kMaxStages + 4 + 2 * kDescRingTC;
+constexpr int kNumBars = 2 * kMaxRawStages + 4 * kMaxStages + 4 + 2 * kDescRingTC;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffRings = 1024;
 static_assert(kOffTmemSlot + 16 <= kOffRings, "fixed part");
@@ -103,28 +103,34 @@ constexpr int kSmemLimit = 232448 - 1024;  // 227 KiB opt-in per CTA, minus stat
 // Ring geometry for a launch whose largest MMA N is nmax (each CTA holds nmax/2 rows x
 // kBChunks chunks of a B stage). A and B stages both cover one 128-wide K step.
 struct TcRings {
-  int a_stages, b_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
+  int a_stages, b_stages, raw_stages, b_stage_bytes, off_a, off_b, off_raw, smem_bytes;
 };
 __host__ __device__ inline TcRings tc_rings(int nmax) {
   auto clamp = [](int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); };
   TcRings r;
   r.b_stage_bytes = (nmax / 2) * 128 * kBChunks;
-  const int avail = kSmemLimit - 1024 - kOffRings - kRawStages * kRawStageBytes;
-  // enough activation stages to cover the L2 latency, then as deep an A ring as fits
-  // (the dequant warps run ahead of the MMA), then whatever is left back to B
+  const int avail = kSmemLimit - 1024 - kOffRings;
+  // enough activation stages to cover the L2 latency and a two-deep A ring; then as many
+  // raw weight stages as fit (the weight copies wait on HBM, so with small activation
+  // tiles the spare room goes to weights in flight); then what is left to A, then B gets
+  // what remains (fewer stages than the latency target when the tiles are large)
   int bs = clamp((kBInFlightBytes + r.b_stage_bytes - 1) / r.b_stage_bytes, 2, kMaxStages);
-  const int as = clamp((avail - bs * r.b_stage_bytes) / kAStageBytes, 2, kMaxStages);
-  bs = clamp((avail - as * kAStageBytes) / r.b_stage_bytes, bs, kMaxStages);
+  const int rs = clamp((avail - bs * r.b_stage_bytes - 2 * kAStageBytes) / kRawStageBytes, 3, kMaxRawStages);
+  const int as = clamp((avail - bs * r.b_stage_bytes - rs * kRawStageBytes) / kAStageBytes, 2, kMaxStages);
+  bs = clamp((avail - as * kAStageBytes - rs * kRawStageBytes) / r.b_stage_bytes, 2, kMaxStages);
   r.a_stages = as;
   r.b_stages = bs;
+  r.raw_stages = rs;
   r.off_a = kOffRings;
   r.off_b = r.off_a + as * kAStageBytes;
   r.off_raw = r.off_b + bs * r.b_stage_bytes;
-  r.smem_bytes = r.off_raw + kRawStages * kRawStageBytes + 1024;  // + base alignment slack
+  r.smem_bytes = r.off_raw + rs * kRawStageBytes + 1024;  // + base alignment slack
   return r;
 }
 
-enum Epi { kGateUp = 0, kDown = 1 };
+// kGateUp: SiLU(gate) * up into a; kDown: fp32 y by position; kPlain: bf16 out[row, n]
+// (grouped operators).
+enum Epi { kGateUp = 0, kDown = 1, kPlain = 2 };
 
 // Position in a ring of runtime size: slot index and the phase parity of its barriers.
 struct RingPos {
@@ -149,6 +155,8 @@ struct TcParams {
   int64_t n_slots;
   int topk;
   int64_t cap;
+  const int32_t* block_row0;  // activation row of each block's first position (grouped), or null
+  uint16_t* out;              // kPlain output [rows, N]
   uint16_t* a_out;
   float* y_out;
   const float* topk_weights;
@@ -192,6 +200,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   const int AS = p.rings.a_stages, BS = p.rings.b_stages;
+  const uint32_t RS = uint32_t(p.rings.raw_stages);
   const int DS = AS > BS ? AS : BS;  // depth of the step barrier ring
   const int b_stage_bytes = p.rings.b_stage_bytes;
   const uint32_t rank = cluster_rank();
@@ -199,8 +208,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* raw_full = bars;
-  uint64_t* raw_empty = raw_full + kRawStages;
-  uint64_t* step_full = raw_empty + kRawStages;  // [D] used in rank 0: dequant arrivals + copies
+  uint64_t* raw_empty = raw_full + kMaxRawStages;
+  uint64_t* step_full = raw_empty + kMaxRawStages;  // [D] used in rank 0: dequant arrivals + copies
   uint64_t* step_empty = step_full + kMaxStages; // [D] one multicast commit per step
   uint64_t* spare = step_empty + kMaxStages;     // [2 * kMaxStages] unused
   uint64_t* acc_full = spare + 2 * kMaxStages;   // [2]
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       abort_flag = 2;
       if (blockIdx.x == 0) atomicOr(p.status, CHORD_DEV_BLOB_MISMATCH);
     }
-    for (int s = 0; s < kRawStages; ++s) {
+    for (int s = 0; s < p.rings.raw_stages; ++s) {
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kDequantWarps);
     }
@@ -269,13 +278,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     // routing metadata of item w (its expert and the flat slots of this lane's 8 rows),
     // loaded one item ahead so the latency overlaps the current item's streaming
-    auto load_meta = [&](int64_t w, int& e, int (&f)[kMaxN / 32]) {
+    auto load_meta = [&](int64_t w, int& e, int& r0, int (&f)[kMaxN / 32]) {
       e = -1;
+      r0 = 0;
 #pragma unroll
       for (int i = 0; i < kMaxN / 32; ++i) f[i] = -1;
       if (w >= items) return;
       const int64_t b = w / NT2;
       e = __ldg(p.expert_ids + b);
+      r0 = p.block_row0 ? __ldg(p.block_row0 + b) : int(b * p.block_m);
       const int pos0 = int(b * p.block_m);
 #pragma unroll
       for (int i = 0; i < kMaxN / 32; ++i) {
@@ -283,15 +294,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (r < p.block_m) f[i] = __ldg(p.sorted_ids + pos0 + r);
       }
     };
-    int e_next, f_next[kMaxN / 32];
-    load_meta(cid, e_next, f_next);
+    int e_next, r0_next, f_next[kMaxN / 32];
+    load_meta(cid, e_next, r0_next, f_next);
     for (int64_t w = cid; ok; w += ncl) {
       const bool end = w >= items;
       int e = e_next, nt = 0, pos0 = 0, nvalid = 0;
+      const int r0 = r0_next;
       int fcur[kMaxN / 32];
 #pragma unroll
       for (int i = 0; i < kMaxN / 32; ++i) fcur[i] = f_next[i];
-      load_meta(w + ncl, e_next, f_next);
+      load_meta(w + ncl, e_next, r0_next, f_next);
       if (!end) {
         nt = int(w % NT2) * 2 + int(rank);
         pos0 = int((w / NT2) * p.block_m);
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int nmma = (nvalid + 15) & ~15;
       const int half = nmma >> 1;                 // rows per CTA, a multiple of 8
       const CUtensorMap* map = &maps.m[(half >> 3) - 1];
-      const int row0 = pos0 + int(rank) * half;
+      const int row0 = r0 + int(rank) * half;
       for (int kb = 0; kb < KT; ++kb) {
         const uint32_t s = bpos.slot;
         // the slot's previous fill (BS steps ago) must have been consumed
@@ -376,9 +388,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       for (int kt0 = 0; kt0 < KT; kt0 += kRawTiles) {
         const int ntl = min(kRawTiles, KT - kt0);
-        const uint32_t rs = rstage % kRawStages;
-        if (rstage >= uint32_t(kRawStages) &&
-            !mbar_wait(&raw_empty[rs], ((rstage / kRawStages) - 1) & 1, abort_v, p.status)) {
+        const uint32_t rs = rstage % RS;
+        if (rstage >= RS && !mbar_wait(&raw_empty[rs], ((rstage / RS) - 1) & 1, abort_v, p.status)) {
           ok = false;
           break;
         }
@@ -400,8 +411,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // drain: wait (bounded, ignoring abort) for the copies still in flight
     if (lane == 0) {
       int dummy = 0;
-      for (uint32_t s = (rstage > uint32_t(kRawStages) ? rstage - kRawStages : 0); s < rstage; ++s)
-        mbar_wait(&raw_full[s % kRawStages], (s / kRawStages) & 1, &dummy, p.status);
+      for (uint32_t s = (rstage > RS ? rstage - RS : 0); s < rstage; ++s)
+        mbar_wait(&raw_full[s % RS], (s / RS) & 1, &dummy, p.status);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA issuer
@@ -475,8 +486,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       for (int kt0 = 0; kt0 < KT && ok; kt0 += kRawTiles) {
         const int ntl = min(kRawTiles, KT - kt0);
-        const uint32_t rs = rstage % kRawStages;
-        if (!mbar_wait(&raw_full[rs], (rstage / kRawStages) & 1, abort_v, p.status)) { ok = false; break; }
+        const uint32_t rs = rstage % RS;
+        if (!mbar_wait(&raw_full[rs], (rstage / RS) & 1, abort_v, p.status)) { ok = false; break; }
         const uint32_t raw = sbase + p.rings.off_raw + rs * kRawStageBytes;
         for (int tl = 0; tl < ntl; ++tl) {
           // this lane's share of the tile: four code words and four group scales of its row
@@ -560,6 +571,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (gate && f >= 0)
                 p.a_out[int64_t(d.pos0 + c0 + c) * p.I + i_col] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(v[c], u)));
+            }
+          } else if (EPI == kPlain) {
+            // out[row, n]: a warp stores 32 neighbouring columns (64 bytes) of one row
+            const int n_col = d.nt * kTileN + r;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int f = __shfl_sync(0xffffffffu, f_set, (c0 & 31) + c);
+              if (f >= 0)
+                p.out[int64_t(f) * p.N + n_col] = __bfloat16_as_ushort(__float2bfloat16_rn(v[c]));
             }
           } else {
             // y by sorted position in 128-column blocks: this item's tile is one
@@ -757,6 +777,31 @@ cudaError_t launch_tc_gemms(const ForwardArgs& a, cudaStream_t stream, cudaEvent
   p.K = a.I;
   p.role = CHORD_ROLE_DOWN;
   return launch_one<kDown>(maps, p, grid, stream);
+}
+
+cudaError_t launch_tc_grouped(const GroupedArgs& g, cudaStream_t stream) {
+  TcParams p{};
+  p.sorted_ids = g.sorted_ids;
+  p.expert_ids = g.expert_ids;
+  p.block_row0 = g.block_row0;
+  p.ntp = g.ntp;
+  p.block_m = g.bm;
+  p.n_slots = g.rows;  // sorted_ids holds x rows
+  p.topk = 1;
+  p.cap = g.cap;
+  p.out = g.out;
+  p.E = g.E;
+  p.status = g.status;
+  p.rings = tc_rings(min(kMaxN, g.bm));
+  p.blob = g.w;
+  p.tiles = g.w + blob_tiles_offset();
+  p.N = g.N;
+  p.K = g.K;
+  p.role = g.role;
+  BoxMaps maps;
+  cudaError_t err = box_maps(&maps, g.x, g.rows, g.K);
+  if (err != cudaSuccess) return err;
+  return launch_one<kPlain>(maps, p, g.num_sms, stream);
 }
 
 }  // namespace chord
