@@ -10,7 +10,9 @@
 //                 tile nt) two at a time, publishes both descriptors, then streams the two
 //                 items' stages alternately, each stage ONE bulk copy of KTS consecutive
 //                 128-wide K tiles (codes + scales, up to 36 KiB: a bulk copy has a high fixed
-//                 cost, so bytes per copy decide the streaming rate). The few routed
+//                 cost, so bytes per copy decide the streaming rate). When K is shorter than
+//                 a stage (K = 256 of the TP8 down projection), an item spans several
+//                 adjacent 128-row tiles so that its one copy is still full. The few routed
 //                 activation rows are small and shared by every warp, so consumers read them
 //                 straight from global memory through L1 (ld.global.nc) instead of staging them.
 //   warps 1..8    consumer group 0 takes the first item of each pair, warps 9..16 group 1
@@ -85,10 +87,6 @@ __device__ __forceinline__ uint4 ldg_nc128(const void* p) {
   return v;
 }
 
-// Dequantises NTILE tiles of a stage (tiles t0, t0 + 2, ...) for warp `rb` (16 rows) and
-// accumulates them against the routed activation rows (xrow[n8] points at this lane's row
-// of 8-token tile n8, advanced to the stage's first K): the A fragments of
-// mma.m16n8k16 come straight out of dequant8; tokens are the N dimension.
 // This warp's code words (rows g and g + 8 of its 16-row block) and scales of one tile.
 struct TileCodes {
   uint4 c0, c1, sv;
@@ -102,51 +100,48 @@ __device__ __forceinline__ TileCodes load_tile_codes(const uint8_t* stg, int til
   return tc;
 }
 
-template <int NT8, int NSET, int NTILE, class S>
-__device__ __forceinline__ void consume_tiles(const TileCodes (&codes)[NTILE], int t0, int lane,
-                                              const uint16_t* const (&xrow)[NT8],
-                                              float (&acc)[NT8][NSET][4], int chain0) {
-  const int t = lane & 3;
-  uint4 c0[NTILE], c1[NTILE], sv[NTILE];
+// The activation fragments of one 128-K tile: K step j (32 K) of 8-token tile n8, this
+// lane's 8 consecutive K of its token row. xrow[n8] points at the lane's row, already
+// offset by 8 * (lane % 4); `off` is the tile's first K.
+template <int NT8>
+__device__ __forceinline__ void load_tile_x(uint4 (&xv)[4][NT8], const uint16_t* const (&xrow)[NT8], int off) {
 #pragma unroll
-  for (int u = 0; u < NTILE; ++u) {
-    c0[u] = codes[u].c0;
-    c1[u] = codes[u].c1;
-    sv[u] = codes[u].sv;
-  }
-  // the tile's activation fragments, issued together ahead of the dequantisation so their
-  // L1 latency overlaps it
-  uint4 xv[NTILE][4][NT8];
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-  for (int u = 0; u < NTILE; ++u)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) xv[u][j][n8] = ldg_nc128(xrow[n8] + (t0 + 2 * u) * kTileK + 32 * j + 8 * t);
+    for (int n8 = 0; n8 < NT8; ++n8) xv[j][n8] = ldg_nc128(xrow[n8] + off + 32 * j);
+}
+
+// Dequantises one tile for warp `rb` (16 rows) and accumulates it against the routed
+// activation rows: the A fragments of mma.m16n8k16 come straight out of dequant8; tokens
+// are the N dimension. xv holds the tile's activation fragments, loaded at the tile's
+// start so that their latency overlaps the first dequantisation. (Refilling each K step's
+// fragments with the next tile's right after its MMAs, a whole tile ahead, cut the
+// long-scoreboard stalls but measured 3% slower.)
+template <int NT8, int NSET>
+__device__ __forceinline__ void consume_tile(const TileCodes& code, const uint4 (&xv)[4][NT8],
+                                             float (&acc)[NT8][NSET][4], int chain0) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    const uint32_t cw0 = j == 0 ? code.c0.x : j == 1 ? code.c0.y : j == 2 ? code.c0.z : code.c0.w;
+    const uint32_t cw1 = j == 0 ? code.c1.x : j == 1 ? code.c1.y : j == 2 ? code.c1.z : code.c1.w;
+    // scale pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
+    const uint32_t sp0 = (j >> 1) ? code.sv.y : code.sv.x;
+    const uint32_t sp1 = (j >> 1) ? code.sv.w : code.sv.z;
+    uint32_t w0[4], w1[4];
+    dequant8(cw0, bf16_splat_half(sp0, j & 1), w0);
+    dequant8(cw1, bf16_splat_half(sp1, j & 1), w1);
+    const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
+    const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
 #pragma unroll
-    for (int u = 0; u < NTILE; ++u) {
-      const uint32_t cw0 = j == 0 ? c0[u].x : j == 1 ? c0[u].y : j == 2 ? c0[u].z : c0[u].w;
-      const uint32_t cw1 = j == 0 ? c1[u].x : j == 1 ? c1[u].y : j == 2 ? c1[u].z : c1[u].w;
-      // scale pairs: (h0 j0,j1) (h0 j2,j3) (h1 j0,j1) (h1 j2,j3)
-      const uint32_t sp0 = (j >> 1) ? sv[u].y : sv[u].x;
-      const uint32_t sp1 = (j >> 1) ? sv[u].w : sv[u].z;
-      uint32_t w0[4], w1[4];
-      dequant8(cw0, bf16_splat_half(sp0, j & 1), w0);
-      dequant8(cw1, bf16_splat_half(sp1, j & 1), w1);
-      const uint32_t a_lo[4] = {w0[0], w1[0], w0[1], w1[1]};
-      const uint32_t a_hi[4] = {w0[2], w1[2], w0[3], w1[3]};
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) {
-        mma_bf16_16816(acc[n8][(chain0 + 2 * u) % NSET], a_lo, xv[u][j][n8].x, xv[u][j][n8].y);
-        mma_bf16_16816(acc[n8][(chain0 + 2 * u + 1) % NSET], a_hi, xv[u][j][n8].z, xv[u][j][n8].w);
-      }
+    for (int n8 = 0; n8 < NT8; ++n8) {
+      mma_bf16_16816(acc[n8][chain0 % NSET], a_lo, xv[j][n8].x, xv[j][n8].y);
+      mma_bf16_16816(acc[n8][(chain0 + 1) % NSET], a_hi, xv[j][n8].z, xv[j][n8].w);
     }
   }
 }
 
-template <int EPI, int TC>
+// MULTI: the item covers NTPI > 1 tiles of 128 rows (a K shorter than a stage, see NTPI)
+template <int EPI, int TC, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p) {
   using S = Smem<TC>;
   constexpr int NT8 = TC / 8;
@@ -188,8 +183,19 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
   volatile int* abort_v = &abort_flag;
 
   const int KT = p.K / kTileK;
-  const int KS = (KT + KTS - 1) / KTS;         // stages per item
   const int NTILES = p.N / kTileN;
+  // With a short K (KT < KTS) one tile's K would fill only part of a stage, and a bulk
+  // copy's fixed cost makes small copies slow; an item then covers NTPI consecutive
+  // 128-row tiles of its expert (adjacent in the blob), so one copy still carries up to
+  // KTS tiles. NTPI divides NTILES.
+  int NTPI = 1;
+  if (MULTI && KT < KTS) {
+    NTPI = KTS / KT;
+    while (NTILES % NTPI) --NTPI;
+  }
+  const int KTI = KT * NTPI;                   // tiles per item
+  const int KS = (KTI + KTS - 1) / KTS;        // stages per item
+  const int NGRP = NTILES / NTPI;              // items per routing chunk
   const int cpb = (p.block_m + TC - 1) / TC;  // token chunks per routing block
 
   if (warp == 0) {
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     if (ntp < 0) ntp = 0;
     if (ntp > p.cap) ntp = int(p.cap);
     const int64_t nblocks = ntp / p.block_m;
-    const int64_t items = nblocks * cpb * NTILES;
+    const int64_t items = nblocks * cpb * NGRP;
     const uint64_t pol_w = policy_evict_first();
     uint32_t stage = 0;      // global stage counter
     uint32_t nitem = 0;      // published descriptors
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       pos0 = 0;
       f = -1;
       if (w >= items) return;
-      const int64_t bc = w / NTILES;
+      const int64_t bc = w / NGRP;
       const int64_t b = bc / cpb;
       const int c = int(bc % cpb);
       e = __ldg(p.expert_ids + b);
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
         e = qe[0];
         pos0 = qpos[0];
         fval = qf[0];
-        nt = int(w % NTILES);
+        nt = int(w % NGRP);
 #pragma unroll
         for (int i = 0; i + 1 < kLook; ++i) {
           qe[i] = qe[i + 1];
@@ -268,10 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
           !mbar_wait(&empty[slot], ((stage / NSTAGE) - 1) & 1, abort_v, p.status))
         return false;
       const int kt0 = ks * KTS;
-      const int ntl = min(KTS, KT - kt0);
+      const int ntl = min(KTS, KTI - kt0);
       if (lane == 0) {
         uint8_t* st = stages + slot * S::kStageBytes;
-        const uint64_t tile0 = (uint64_t(e) * NTILES + nt) * KT;
+        const uint64_t tile0 = (uint64_t(e) * NTILES + uint64_t(nt) * NTPI) * KT;
         mbar_arrive_expect_tx(&full[slot], uint32_t(ntl) * kTileBytes);
         bulk_g2s_hint(st, p.tiles + (tile0 + kt0) * kTileBytes, uint32_t(ntl) * kTileBytes, &full[slot], pol_w);
       }
@@ -334,94 +340,110 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 #pragma unroll
       for (int q = 0; q < NSET; ++q) acc[i][q][0] = acc[i][q][1] = acc[i][q][2] = acc[i][q][3] = 0.f;
 
+    // this lane's 8 K of each row
+    const uint16_t* xrow[NT8];
+#pragma unroll
+    for (int n8 = 0; n8 < NT8; ++n8) xrow[n8] = xrow0[n8] + 8 * t;
+
+    // ---- epilogue of 128-row tile `ntile` (the item's last, or with a short K each of its
+    // NTPI tiles in turn, leaving the accumulators zeroed for the next)
+    auto epilogue = [&](int ntile) {
+      float accs[NT8][4];
+#pragma unroll
+      for (int i = 0; i < NT8; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v = 0.f;
+#pragma unroll
+          for (int q = 0; q < NSET; ++q) {
+            v += acc[i][q][c];
+            if (MULTI) acc[i][q][c] = 0.f;
+          }
+          accs[i][c] = v;
+        }
+      if (EPI == kGateUp) {
+        const int i_col = ntile * (kTileN / 2) + rb * 8 + g;  // intermediate column
+#pragma unroll
+        for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int col = n8 * 8 + 2 * t + q;
+            if (d.f[col] >= 0) {
+              const float v = silu_mul(accs[n8][q], accs[n8][2 + q]);
+              p.a_out[int64_t(d.pos0 + col) * p.I + i_col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
+          }
+        }
+      } else if (EPI == kPlain) {
+        const int n0 = ntile * kTileN + rb * 16 + g;
+#pragma unroll
+        for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int f = d.f[n8 * 8 + 2 * t + q];
+            if (f >= 0) {
+              uint16_t* orow = p.out + int64_t(f) * p.N;
+              orow[n0] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][q]));
+              orow[n0 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][2 + q]));
+            }
+          }
+        }
+      } else {
+        const int n0 = ntile * kTileN + rb * 16 + g;
+#pragma unroll
+        for (int n8 = 0; n8 < NT8; ++n8) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int col = n8 * 8 + 2 * t + q;
+            const int f = d.f[col];
+            if (f >= 0) {
+              float* yr = p.y_out + int64_t(f) * p.H;
+              yr[n0] = accs[n8][q];
+              yr[n0 + 8] = accs[n8][2 + q];
+            }
+          }
+        }
+      }
+    };
+
     const uint32_t s0 = d.s0;
     const int sstride = d.sstride;
+    int kt = 0, sub = 0;  // MULTI: K tile inside the current 128-row tile, and that tile's index
     for (int ks = 0; ks < KS; ++ks) {
       const uint32_t s = s0 + uint32_t(ks * sstride);
       const uint32_t slot = s % NSTAGE;
       if (!mbar_wait(&full[slot], (s / NSTAGE) & 1, abort_v, p.status)) return;
-      const int ntl = min(KTS, KT - ks * KTS);
+      const int ntl = min(KTS, KTI - ks * KTS);
       // plain shared loads (ordered after the wait by its memory clobber) so the compiler
       // can schedule them ahead of the dequantisation and the MMAs
       const uint8_t* stg = stages + slot * S::kStageBytes;
-      const uint16_t* xrow[NT8];
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) xrow[n8] = xrow0[n8] + ks * KTS * kTileK;
       // software-pipelined over the stage's tiles: tile i + 1's codes are loaded from shared
       // memory before tile i is dequantised, so their latency overlaps the math
-      TileCodes cur[1] = {load_tile_codes(stg, 0, rb, lane)};
+      TileCodes cur = load_tile_codes(stg, 0, rb, lane);
       for (int i = 0; i < ntl; ++i) {
-        TileCodes nxt = cur[0];
+        TileCodes nxt = cur;
         if (i + 1 < ntl) nxt = load_tile_codes(stg, i + 1, rb, lane);
-        consume_tiles<NT8, NSET, 1, S>(cur, i, lane, xrow, acc, (i & 1) * 2);
-        cur[0] = nxt;
+        uint4 xv[4][NT8];
+        load_tile_x<NT8>(xv, xrow, (MULTI ? kt : ks * KTS + i) * kTileK);
+        consume_tile<NT8, NSET>(cur, xv, acc, (i & 1) * 2);
+        cur = nxt;
+        if (MULTI && ++kt == KT) {
+          kt = 0;
+          if (++sub < NTPI) epilogue(d.nt * NTPI + sub - 1);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    float accs[NT8][4];
-#pragma unroll
-    for (int i = 0; i < NT8; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v = 0.f;
-#pragma unroll
-        for (int q = 0; q < NSET; ++q) v += acc[i][q][c];
-        accs[i][c] = v;
-      }
-
-    // ---- epilogue (this group's item)
-    if (EPI == kGateUp) {
-      const int i_col = d.nt * (kTileN / 2) + rb * 8 + g;  // intermediate column
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) {
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int col = n8 * 8 + 2 * t + q;
-          if (d.f[col] >= 0) {
-            const float v = silu_mul(accs[n8][q], accs[n8][2 + q]);
-            p.a_out[int64_t(d.pos0 + col) * p.I + i_col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-          }
-        }
-      }
-    } else if (EPI == kPlain) {
-      const int n0 = d.nt * kTileN + rb * 16 + g;
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) {
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int f = d.f[n8 * 8 + 2 * t + q];
-          if (f >= 0) {
-            uint16_t* orow = p.out + int64_t(f) * p.N;
-            orow[n0] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][q]));
-            orow[n0 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(accs[n8][2 + q]));
-          }
-        }
-      }
-    } else {
-      const int n0 = d.nt * kTileN + rb * 16 + g;
-#pragma unroll
-      for (int n8 = 0; n8 < NT8; ++n8) {
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int col = n8 * 8 + 2 * t + q;
-          const int f = d.f[col];
-          if (f >= 0) {
-            float* yr = p.y_out + int64_t(f) * p.H;
-            yr[n0] = accs[n8][q];
-            yr[n0 + 8] = accs[n8][2 + q];
-          }
-        }
-      }
-    }
+    epilogue(d.nt * NTPI + NTPI - 1);
     __syncwarp();
     if (lane == 0) mbar_arrive(&dempty[ds]);
   }
 }
 
-template <int EPI, int TC>
+template <int EPI, int TC, bool MULTI>
 cudaError_t launch_one(const StreamParams& p, int grid, cudaStream_t stream) {
-  auto kern = stream_gemm_kernel<EPI, TC>;
+  auto kern = stream_gemm_kernel<EPI, TC, MULTI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Smem<TC>::kBytes);
   if (err != cudaSuccess) return err;
@@ -430,13 +452,20 @@ cudaError_t launch_one(const StreamParams& p, int grid, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int EPI, bool MULTI>
+cudaError_t launch_tc_m(const StreamParams& p, int tc, int grid, cudaStream_t stream) {
+  switch (tc) {
+    case 8: return launch_one<EPI, 8, MULTI>(p, grid, stream);
+    case 16: return launch_one<EPI, 16, MULTI>(p, grid, stream);
+    default: return launch_one<EPI, 32, MULTI>(p, grid, stream);
+  }
+}
+
 template <int EPI>
 cudaError_t launch_tc(const StreamParams& p, int tc, int grid, cudaStream_t stream) {
-  switch (tc) {
-    case 8: return launch_one<EPI, 8>(p, grid, stream);
-    case 16: return launch_one<EPI, 16>(p, grid, stream);
-    default: return launch_one<EPI, 32>(p, grid, stream);
-  }
+  // a K shorter than one stage's 4 tiles takes the multi-tile item variant
+  return p.K < 4 * kTileK ? launch_tc_m<EPI, true>(p, tc, grid, stream)
+                          : launch_tc_m<EPI, false>(p, tc, grid, stream);
 }
 
 }  // namespace
