@@ -40,7 +40,11 @@ def invert_layout(blob: np.ndarray, E, N, K, role):
     NT, KT = N // 128, K // 128
     tiles = blob[256:256 + E * NT * KT * 9216].reshape(E, NT, KT, 9216)
     codes = np.ascontiguousarray(tiles[..., :8192]).view(np.uint32)
-    codes = codes.reshape(E, NT, KT, 8, 2, 8, 4, 4)          # e nt kt rb h g t j
+    codes = codes.reshape(E, NT, KT, 8, 2, 8, 4, 4)          # e nt kt rb h g slot j
+    # the 16-byte vector of K slice t of row g sits in slot t ^ ((g >> 1) & 3)
+    g = np.arange(8)[:, None].repeat(4, axis=1)
+    t = np.arange(4)[None, :].repeat(8, axis=0)
+    codes = codes[..., g, t ^ ((g >> 1) & 3), :]             # e nt kt rb h g t j
     # un-permute nibbles: K offset u sits in nibble (u>>1) + 4*(u&1)
     slot = [(u >> 1) + 4 * (u & 1) for u in range(8)]
     words = np.zeros(codes.shape, dtype=np.uint32)
@@ -70,7 +74,7 @@ def test_repack_layout_round_trip(chord, role, E, N, K):
     s = rng.integers(0, 2 ** 16, size=(E, N, K // 32), dtype=np.uint16)
     blob = repack(chord, qw, s, role).cpu().numpy()
     hdr = blob[:48].view(np.uint32)
-    assert hdr[0] == 0x34574843 and hdr[1] == 2 and hdr[2] == 2 and hdr[3] == role
+    assert hdr[0] == 0x34574843 and hdr[1] == 3 and hdr[2] == 2 and hdr[3] == role
     assert list(hdr[4:8].view(np.int32)) == [E, N, K, 32]
     qw2, s2 = invert_layout(blob, E, N, K, role)
     assert np.array_equal(qw2, qw)

@@ -12,10 +12,13 @@
 //
 // Codes: 8 sub-tiles of 16 rows (rb = 0..7, 1 KiB each). Inside a sub-tile the int32
 // word index is
-//     h*128 + g*16 + t*4 + j         (h 0..1, g 0..7, t 0..3, j 0..3)
+//     h*128 + g*16 + code_slot(g, t)*4 + j      (h 0..1, g 0..7, t 0..3, j 0..3)
 // and holds physical row  rb*16 + 8h + g  and K range  kt*128 + 32j + 8t + [0, 8).
-// Lane (g, t) of a warp therefore reads its two 16-byte vectors (h = 0, 1) from
-// contiguous 512-byte spans. Inside a word, K offset u (0..7) sits in nibble
+// code_slot(g, t) = t ^ ((g >> 1) & 3) swizzles the four 16-byte vectors of a row so
+// that both ways of reading a sub-tile half are free of shared-memory bank conflicts:
+// lane (g, t) of a warp reading its vector (weight streaming: 8 lanes of a phase cover
+// one contiguous 128-byte span), and lane = row with t fixed across the warp (tensor core:
+// 8 consecutive rows land in 8 distinct 16-byte bank groups). Inside a word, K offset u (0..7) sits in nibble
 // (u >> 1) + 4 * (u & 1), so that masking nibbles {i, i+4} after a right shift by 4i
 // yields the bf16 pair (u = 2i, 2i+1) in order.
 //
@@ -37,7 +40,7 @@
 namespace chord {
 
 constexpr uint32_t kBlobMagic = 0x34574843u;  // "CHW4"
-constexpr uint32_t kBlobVersion = 2;
+constexpr uint32_t kBlobVersion = 3;
 constexpr uint32_t kLayoutTile128 = 2;  // 128x128 tiles, scales interleaved after codes
 constexpr int kGroup = 32;
 constexpr int kTileN = 128;
@@ -76,6 +79,9 @@ __host__ __device__ inline int logical_row(int role, int N, int p) {
   int blk = p >> 4, r = p & 15;
   return r < 8 ? (blk * 8 + r) : (N / 2 + blk * 8 + (r - 8));
 }
+
+// 16-byte vector slot (0..3) of K slice t of sub-tile row g (see the layout above).
+__host__ __device__ inline int code_slot(int g, int t) { return t ^ ((g >> 1) & 3); }
 
 // Nibble slot holding K offset u (0..7) of a repacked word.
 __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1); }

@@ -36,7 +36,8 @@ __global__ void repack_codes_kernel(const int32_t* __restrict__ qweight, int E, 
     const int n = logical_row(role, N, p);
     const int k0 = kt * kTileK + 32 * j + 8 * t;
     const uint32_t src = uint32_t(qweight[(int64_t(e) * N + n) * (K / 8) + k0 / 8]);
-    reinterpret_cast<uint32_t*>(tiles + tile * kTileBytes)[w & 2047] = permute_nibbles(src);
+    const int dst = rb * 256 + h * 128 + g * 16 + code_slot(g, t) * 4 + j;
+    reinterpret_cast<uint32_t*>(tiles + tile * kTileBytes)[dst] = permute_nibbles(src);
   }
 }
 
@@ -101,7 +102,8 @@ __global__ void dequant_blob_kernel(const uint8_t* __restrict__ blob, int E, int
     const uint8_t* tp = tiles + tile * kTileBytes;
     const uint16_t s = reinterpret_cast<const uint16_t*>(tp + kTileCodeBytes)[rb * 64 + g * 8 + h * 4 + j];
     uint32_t pairs[4];
-    dequant8(reinterpret_cast<const uint32_t*>(tp)[i & 2047], bf16_splat(s), pairs);
+    dequant8(reinterpret_cast<const uint32_t*>(tp)[rb * 256 + h * 128 + g * 16 + code_slot(g, t) * 4 + j],
+             bf16_splat(s), pairs);
     uint4 v = make_uint4(pairs[0], pairs[1], pairs[2], pairs[3]);
     *reinterpret_cast<uint4*>(w + (int64_t(e) * N + n) * K + k0) = v;
   }

@@ -93,9 +93,10 @@ struct TileCodes {
 };
 __device__ __forceinline__ TileCodes load_tile_codes(const uint8_t* stg, int tile, int rb, int lane) {
   const uint8_t* st = stg + tile * kTileBytes;
+  const int g = lane >> 2, v = g * 16 + code_slot(g, lane & 3) * 4;  // this lane's vector (in words)
   TileCodes tc;
-  tc.c0 = *reinterpret_cast<const uint4*>(st + rb * 1024 + lane * 16);
-  tc.c1 = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + lane * 16);
+  tc.c0 = *reinterpret_cast<const uint4*>(st + rb * 1024 + v * 4);
+  tc.c1 = *reinterpret_cast<const uint4*>(st + rb * 1024 + 512 + v * 4);
   tc.sv = *reinterpret_cast<const uint4*>(st + kTileCodeBytes + rb * 128 + (lane >> 2) * 16);
   return tc;
 }

@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int tl = 0; tl < ntl; ++tl) {
           // this lane's share of the tile: four code words and four group scales of its row
           const uint32_t tb = raw + tl * kTileBytes;
-          const uint4 c = lds128(tb + rb * 1024 + hrow * 512 + g * 64 + t * 16);
+          const uint4 c = lds128(tb + rb * 1024 + hrow * 512 + g * 64 + code_slot(g, t) * 16);
           const uint2 sc = lds64(tb + kTileCodeBytes + rb * 128 + g * 16 + hrow * 8);
           const uint32_t s = apos.slot;
           // the slot's previous fill (AS steps ago) must have been consumed
