@@ -14,7 +14,11 @@
 //   n <= 4 x 1024  : one CTA of 32 warps (runs of ceil(n/1024) steps) does count, scan,
 //                    scatter and fill (1 launch)
 //   larger n       : count kernel (per-chunk histograms) -> scan kernel (1 CTA) ->
-//                    scatter + fill kernel, histograms in the caller's workspace.
+//                    scatter + fill kernel, histograms in the caller's workspace. A chunk
+//                    (one warp's run) is 256 slots, so a prefill batch spreads over
+//                    hundreds of warps, unless E x chunks would pass 2^17 histogram
+//                    entries; then it is 1024 slots (the workspace stays within what the
+//                    no-allocation variant's static scratch holds).
 #include <math.h>
 
 #include "chord_internal.cuh"
@@ -22,8 +26,16 @@
 namespace chord {
 namespace {
 
-constexpr int kChunk = 1024;       // flat slots per warp chunk
+constexpr int kChunk = 1024;       // flat slots per warp chunk (largest)
 constexpr int kSteps = kChunk / 32;
+constexpr int kChunkSmall = 256;   // multi-CTA path, when the histograms stay small
+constexpr int64_t kMaxHistEntries = int64_t(1) << 17;
+
+// Slots per warp chunk of the multi-CTA path for n slots and E experts.
+__host__ __device__ inline int multi_chunk(int64_t n, int E) {
+  const int64_t g = (n + kChunkSmall - 1) / kChunkSmall;
+  return int64_t(E) * g <= kMaxHistEntries ? kChunkSmall : kChunk;
+}
 constexpr int kMaxE = 1024;
 // Up to this many 1024-slot chunks the routing sort runs in one CTA (one launch); above
 // it the count / scan / scatter kernels spread the slots over the GPU (one CTA sorting
@@ -342,7 +354,7 @@ __global__ void __launch_bounds__(1024) router_align_single_kernel(
 constexpr int kWarpsPerCta = 4;
 
 __global__ void __launch_bounds__(32 * kWarpsPerCta) align_count_kernel(
-    const int32_t* __restrict__ ids, int64_t n, int E, int64_t G, int* __restrict__ chunk_hist) {
+    const int32_t* __restrict__ ids, int64_t n, int E, int64_t G, int csz, int* __restrict__ chunk_hist) {
   extern __shared__ int smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* row = smem + warp * E;
@@ -351,8 +363,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_count_kernel(
   const int64_t chunk = int64_t(blockIdx.x) * kWarpsPerCta + warp;
   if (chunk >= G) return;
   int v[kSteps];
-  load_steps(ids, n, chunk * kChunk, kSteps, v);
-  chunk_count(v, kSteps, E, key_bits(E), row);
+  load_steps(ids, n, chunk * csz, csz / 32, v);
+  chunk_count(v, csz / 32, E, key_bits(E), row);
   for (int e = lane; e < E; e += 32) chunk_hist[int64_t(e) * G + chunk] = row[e];
 }
 
@@ -364,17 +376,45 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int E, int block_m, in
                                                           int32_t* __restrict__ offsets_out) {
   __shared__ int off[kMaxE + 1];
   __shared__ int wsum[33];
-  const int tid = threadIdx.x;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int run = 0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // a warp per expert: exclusive prefix of its chunk counts over windows of 32 x R chunks,
+  // each lane loading its R consecutive counts at once (one round trip per window)
+  constexpr int R = 8;
+  for (int e = warp; e < E; e += int(blockDim.x >> 5)) {
     int* h = chunk_hist + int64_t(e) * G;
-    for (int64_t g = 0; g < G; ++g) {
-      int c = h[g];
-      h[g] = run;
-      run += c;
+    int run = 0;
+    for (int64_t base = 0; base < G; base += 32 * R) {
+      int c[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int64_t g = base + lane * R + i;
+        c[i] = g < G ? h[g] : 0;
+      }
+      int lsum = 0;
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int x = c[i];
+        c[i] = lsum;
+        lsum += x;
+      }
+      int incl = lsum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      const int excl = run + incl - lsum;
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int64_t g = base + lane * R + i;
+        if (g < G) h[g] = excl + c[i];
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    cnt_g[e] = run;
-    off[e] = (run + block_m - 1) / block_m * block_m;
+    if (lane == 0) {
+      cnt_g[e] = run;
+      off[e] = (run + block_m - 1) / block_m * block_m;
+    }
   }
   __syncthreads();
   const int total = block_exclusive_scan(off, E, wsum);
@@ -391,7 +431,7 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int E, int block_m, in
 
 __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
     const int32_t* __restrict__ ids, int64_t n, int E, int block_m, int64_t G, int64_t cap,
-    int64_t nblocks, const int* __restrict__ chunk_hist, const int* __restrict__ cnt_g,
+    int64_t nblocks, int csz, const int* __restrict__ chunk_hist, const int* __restrict__ cnt_g,
     const int* __restrict__ off_g, int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids) {
   extern __shared__ int smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -401,8 +441,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
     for (int e = lane; e < E; e += 32) row[e] = off_g[e] + chunk_hist[int64_t(e) * G + chunk];
     __syncwarp();
     int v[kSteps];
-    load_steps(ids, n, chunk * kChunk, kSteps, v);
-    chunk_scatter(v, kSteps, chunk * kChunk, E, key_bits(E), row, sorted_ids);
+    load_steps(ids, n, chunk * csz, csz / 32, v);
+    chunk_scatter(v, csz / 32, chunk * csz, E, key_bits(E), row, sorted_ids);
   }
   fill_tail(cnt_g, off_g, E, block_m, n, cap, nblocks, sorted_ids, expert_ids,
             int64_t(blockIdx.x) * blockDim.x + threadIdx.x, int64_t(gridDim.x) * blockDim.x);
@@ -411,16 +451,16 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
 }  // namespace
 
 size_t align_workspace_bytes(int64_t n, int E) {
-  const int64_t G = (n + kChunk - 1) / kChunk;
-  if (G <= kSingleMaxChunks) return 0;
+  if ((n + kChunk - 1) / kChunk <= kSingleMaxChunks) return 0;
+  const int csz = multi_chunk(n, E);
+  const int64_t G = (n + csz - 1) / csz;
   return align256(uint64_t(E) * G * 4) + align256(uint64_t(E) * 4) + align256(uint64_t(E + 1) * 4);
 }
 
 cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int64_t cap,
                          int64_t nblocks, int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntp,
                          int32_t* offsets, void* workspace, cudaStream_t stream) {
-  const int64_t G = (n + kChunk - 1) / kChunk;
-  if (G <= kSingleMaxChunks) {
+  if ((n + kChunk - 1) / kChunk <= kSingleMaxChunks) {
     const size_t smem = (size_t(32) * E + E + E + 1 + 33) * sizeof(int);
     cudaError_t err = cudaFuncSetAttribute(align_single_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -430,6 +470,8 @@ cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int6
     count_launches(1);
     return cudaGetLastError();
   }
+  const int csz = multi_chunk(n, E);
+  const int64_t G = (n + csz - 1) / csz;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* chunk_hist = reinterpret_cast<int*>(ws);
   int* cnt = reinterpret_cast<int*>(ws + align256(uint64_t(E) * G * 4));
@@ -442,10 +484,10 @@ cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int6
   err = cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
   if (err != cudaSuccess) return err;
-  align_count_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem, stream>>>(ids, n, E, G, chunk_hist);
+  align_count_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem, stream>>>(ids, n, E, G, csz, chunk_hist);
   align_scan_kernel<<<1, 1024, 0, stream>>>(E, block_m, G, chunk_hist, cnt, off, ntp, offsets);
   align_scatter_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem, stream>>>(
-      ids, n, E, block_m, G, cap, nblocks, chunk_hist, cnt, off, sorted_ids, expert_ids);
+      ids, n, E, block_m, G, cap, nblocks, csz, chunk_hist, cnt, off, sorted_ids, expert_ids);
   count_launches(3);
   return cudaGetLastError();
 }
