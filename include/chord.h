@@ -291,6 +291,21 @@ CHORD_API chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t 
 CHORD_API chord_status_t chord_set_timing_events(void* const* events, int n);
 CHORD_API uint64_t chord_launch_count(void);
 
+/* ------------------------------------------------------------------------------------
+ * chord_selftest_wait_timeout (diagnostics, no counterpart on the pages): checks the
+ * bounded on-chip wait that every pipeline wait of the GEMM kernels uses, without a
+ * fault. One CTA waits on an mbarrier that nothing ever completes:
+ *   - one thread with a limit of limit_us microseconds (1 .. 1000000): it gives up,
+ *     ORs CHORD_DEV_TIMEOUT into *status and raises the CTA's abort flag;
+ *   - a second thread with the kernels' own limit (1 s): it sees the abort flag and
+ *     returns early, as the other waiters of a GEMM CTA do.
+ * status: device uint32, OR-ed (bit 31 would mean the never-completed phase completed);
+ * elapsed_ns: device uint64[2], the time each of the two threads waited. Asynchronous on
+ * `stream`. Returns CHORD_ERR_INVALID_ARG for null pointers or a limit out of range.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API chord_status_t chord_selftest_wait_timeout(uint32_t* status, uint64_t* elapsed_ns, uint32_t limit_us,
+                                                     chord_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libchord.so")
 SOURCES = ["api.cu", "align.cu", "align_static.cu", "repack.cu", "stream_gemm.cu", "tc_gemm.cu", "permute.cu", "grouped.cu",
-           "combine.cu"]
+           "combine.cu", "diag.cu"]
 HEADERS = ["chord_internal.cuh", "tc_common.cuh"]
 
 NVCC_FLAGS = [

@@ -62,6 +62,7 @@ SIGNATURES = {
     "chord_grouped_masked": (_I, [_P, _I, _I64, _I, _P, _I64, _P, _I, _P, _P, _SZ, _I, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
+    "chord_selftest_wait_timeout": (_I, [_P, _P, ctypes.c_uint32, _P]),
 }
 
 _lib = None
@@ -240,6 +241,12 @@ def chord_set_timing_events(events=None):
 
 def chord_launch_count() -> int:
     return int(lib().chord_launch_count())
+
+
+def chord_selftest_wait_timeout(status, elapsed_ns, limit_us: int, stream=None):
+    """status: int32 device tensor [1] (OR-ed); elapsed_ns: int64 device tensor [2]."""
+    _check(lib().chord_selftest_wait_timeout(_ptr(status), _ptr(elapsed_ns), ctypes.c_uint32(limit_us),
+                                             _stream(stream)), "chord_selftest_wait_timeout")
 
 
 # --------------------------------------------------------------------------- convenience

@@ -469,6 +469,20 @@ chord_status_t chord_set_timing_events(void* const* events, int n) {
 
 uint64_t chord_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+chord_status_t chord_selftest_wait_timeout(uint32_t* status, uint64_t* elapsed_ns, uint32_t limit_us,
+                                           chord_stream_t stream) {
+  g_detail[0] = 0;
+  if (!status || !elapsed_ns) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if (limit_us < 1 || limit_us > 1000000u)
+    return fail(CHORD_ERR_INVALID_ARG, "limit_us must be in [1, 1000000], got %u", limit_us);
+  DeviceInfo dev;
+  chord_status_t st = current_device(&dev);
+  if (st != CHORD_OK) return st;
+  const cudaError_t err = launch_wait_timeout(status, elapsed_ns, uint64_t(limit_us) * 1000ull,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "wait self-test launch");
+}
+
 chord_status_t chord_moe_check_status(void* workspace, chord_stream_t stream_, uint32_t* device_status) {
   g_detail[0] = 0;
   if (!workspace) return fail(CHORD_ERR_INVALID_ARG, "null workspace");

@@ -172,21 +172,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete. Returns false (and raises the CTA's
-// abort flag and the device status) when the wait gave up or another thread aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+// Waits for phase `parity` of `bar` to complete, for at most limit_ns. Returns false (and
+// raises the CTA's abort flag and the device status) when the wait gave up, or false
+// alone when another thread of the CTA had aborted.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                uint32_t* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       if (status) atomicOr(status, CHORD_DEV_TIMEOUT);
       return false;
     }
   }
+}
+
+// The wait every kernel of the library uses: mbar_wait_limit with kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitNs);
 }
 
 // One bulk copy global -> shared, completing `bytes` of transaction on `bar`.
@@ -294,6 +301,8 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 
 // ------------------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files; return cudaGetLastError()).
+
+cudaError_t launch_wait_timeout(uint32_t* status, uint64_t* elapsed_ns, uint64_t limit_ns, cudaStream_t stream);
 
 cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int64_t cap,
                          int64_t nblocks, int32_t* sorted_ids, int32_t* expert_ids,
