@@ -335,6 +335,9 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) ||
                       (!(flags & CHORD_FLAG_FORCE_STREAM) && block_m > 32);
   a.y_blocked = tensor;
+  // early (programmatic) launches on the weight-streaming schedule; not while timing events
+  // are recorded between the kernels (an event between two kernels orders them fully)
+  a.pdl = !tensor && !timing;
   cudaEvent_t mid = timing ? g_timing[1] : nullptr;
   err = tensor ? launch_tc_gemms(a, stream, first, mid) : launch_stream_gemms(a, stream, first, mid);
   if (err != cudaSuccess) return cuda_fail(err, tensor ? "tensor-core GEMM launch" : "streaming GEMM launch");

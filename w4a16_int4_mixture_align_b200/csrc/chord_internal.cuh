@@ -300,6 +300,32 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 }
 
 // ------------------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with launch_pdl may start while the
+// kernel before it on the stream is still running (its CTAs take the SMs the earlier
+// kernel's CTAs leave); it calls grid_dep_wait() before its first access to anything
+// that kernel writes, and grid_dep_wait() returns once that kernel has completed and its
+// memory is visible. grid_dep_trigger() lets this kernel's own dependent launch before
+// this kernel finishes. Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ------------------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files; return cudaGetLastError()).
 
 cudaError_t launch_wait_timeout(uint32_t* status, uint64_t* elapsed_ns, uint64_t limit_ns, cudaStream_t stream);
@@ -335,6 +361,7 @@ struct ForwardArgs {
   uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
   int32_t* slot_pos;  // [T*topk] sorted position of each local flat slot (tensor-core schedule)
   bool y_blocked;     // y is by sorted position in 128-column blocks
+  bool pdl;           // launch the streaming GEMMs and the combine early (programmatic)
   uint32_t* status;
   int64_t T;
   int H, I, E, topk, block_m;

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const int32_t* __restrict__ topk_ids, const float* __restrict__ topk_weights,
     const float* __restrict__ y, const int32_t* __restrict__ slot_pos, uint16_t* __restrict__ out, int64_t T,
     int H, int topk, int E, int64_t cap) {
+  grid_dep_wait();  // launched early: y comes from the down kernel
   const int lane = threadIdx.x & 31;
   const int nchunk = (H + kCombineCols - 1) / kCombineCols;
   for (int64_t item = blockIdx.x; item < T * nchunk; item += gridDim.x) {
@@ -127,14 +128,17 @@ cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
   int64_t grid = a.T * ((a.H + kCombineCols - 1) / kCombineCols);
   if (grid > int64_t(a.num_sms) * 64) grid = int64_t(a.num_sms) * 64;
+  cudaError_t err;
   if (a.y_blocked)
-    combine_kernel<true><<<unsigned(grid), kCombineThreads, 0, stream>>>(
-        a.topk_ids, a.topk_weights, a.y, a.slot_pos, a.out, a.T, a.H, a.topk, a.E, a.cap);
+    err = launch_pdl(a.pdl, combine_kernel<true>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
+                     a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
+                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap);
   else
-    combine_kernel<false><<<unsigned(grid), kCombineThreads, 0, stream>>>(
-        a.topk_ids, a.topk_weights, a.y, a.slot_pos, a.out, a.T, a.H, a.topk, a.E, a.cap);
+    err = launch_pdl(a.pdl, combine_kernel<false>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
+                     a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
+                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap);
   count_launches(1);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_validate(const ForwardArgs& a, cudaStream_t stream) {

@@ -201,6 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
+    // Launched early (programmatic launch), the gate_up kernel may start while the routing
+    // sort still runs: wait for it before reading the routing tensors. The down kernel's
+    // producer reads only those tensors (complete before the gate_up kernel passed this
+    // same wait) and the weights, so it starts streaming at once; its consumers wait for
+    // the intermediate a.
+    if (EPI != kDown) grid_dep_wait();
     int ntp = *p.ntp;
     if (ntp < 0) ntp = 0;
     if (ntp > p.cap) ntp = int(p.cap);
@@ -299,6 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
       }
       if (!has_b) break;
     }
+    // every stage is issued: the next kernel may launch and take SMs as CTAs here finish
+    grid_dep_trigger();
     // end markers at two consecutive indices: one reaches each group
     if (ok) ok = publish(0, 0, 0, -1, true, 0, 1);
     if (ok) publish(0, 0, 0, -1, true, 0, 1);
@@ -313,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
   }
 
   // ------------------------------------------------------------------ consumers
+  if (EPI == kDown) grid_dep_wait();   // the intermediate a comes from the gate_up kernel
   const int cw = warp - 1;             // 0..15
   const int grp = cw >> 3;             // 0 or 1: the first or second item of each pair
   const int rb = cw & 7;               // 16-row block inside the tile
@@ -443,30 +452,30 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
 }
 
 template <int EPI, int TC, bool MULTI>
-cudaError_t launch_one(const StreamParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_one(const StreamParams& p, int grid, bool pdl, cudaStream_t stream) {
   auto kern = stream_gemm_kernel<EPI, TC, MULTI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Smem<TC>::kBytes);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Smem<TC>::kBytes, stream>>>(p);
+  err = launch_pdl(pdl, kern, dim3(grid), dim3(kThreads), size_t(Smem<TC>::kBytes), stream, p);
   count_launches(1);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 template <int EPI, bool MULTI>
-cudaError_t launch_tc_m(const StreamParams& p, int tc, int grid, cudaStream_t stream) {
+cudaError_t launch_tc_m(const StreamParams& p, int tc, int grid, bool pdl, cudaStream_t stream) {
   switch (tc) {
-    case 8: return launch_one<EPI, 8, MULTI>(p, grid, stream);
-    case 16: return launch_one<EPI, 16, MULTI>(p, grid, stream);
-    default: return launch_one<EPI, 32, MULTI>(p, grid, stream);
+    case 8: return launch_one<EPI, 8, MULTI>(p, grid, pdl, stream);
+    case 16: return launch_one<EPI, 16, MULTI>(p, grid, pdl, stream);
+    default: return launch_one<EPI, 32, MULTI>(p, grid, pdl, stream);
   }
 }
 
 template <int EPI>
-cudaError_t launch_tc(const StreamParams& p, int tc, int grid, cudaStream_t stream) {
+cudaError_t launch_tc(const StreamParams& p, int tc, int grid, bool pdl, cudaStream_t stream) {
   // a K shorter than one stage's 4 tiles takes the multi-tile item variant
-  return p.K < 4 * kTileK ? launch_tc_m<EPI, true>(p, tc, grid, stream)
-                          : launch_tc_m<EPI, false>(p, tc, grid, stream);
+  return p.K < 4 * kTileK ? launch_tc_m<EPI, true>(p, tc, grid, pdl, stream)
+                          : launch_tc_m<EPI, false>(p, tc, grid, pdl, stream);
 }
 
 }  // namespace
@@ -500,7 +509,7 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
   p.act_ld = a.H;
   cudaError_t err = first ? record_timing_event(first, stream) : cudaSuccess;
   if (err != cudaSuccess) return err;
-  err = launch_tc<kGateUp>(p, tc, grid, stream);
+  err = launch_tc<kGateUp>(p, tc, grid, a.pdl, stream);
   if (err != cudaSuccess) return err;
   if (mid && (err = record_timing_event(mid, stream)) != cudaSuccess) return err;
 
@@ -512,7 +521,7 @@ cudaError_t launch_stream_gemms(const ForwardArgs& a, cudaStream_t stream, cudaE
   p.role = CHORD_ROLE_DOWN;
   p.act = a.a;
   p.act_ld = a.I;
-  return launch_tc<kDown>(p, tc, grid, stream);
+  return launch_tc<kDown>(p, tc, grid, a.pdl, stream);
 }
 
 cudaError_t launch_stream_grouped(const GroupedArgs& g, cudaStream_t stream) {
@@ -537,7 +546,7 @@ cudaError_t launch_stream_grouped(const GroupedArgs& g, cudaStream_t stream) {
   p.role = g.role;
   p.act = g.x;
   p.act_ld = g.K;
-  return launch_tc<kPlain>(p, tc, g.num_sms, stream);
+  return launch_tc<kPlain>(p, tc, g.num_sms, false, stream);
 }
 
 }  // namespace chord
