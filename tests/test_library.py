@@ -107,3 +107,26 @@ def test_align_rejects_bad_args(lib):
     assert call(f, 16, 2, 2000, 8, f, f, f, None, None, 0, None) == lib.CHORD_ERR_UNSUPPORTED   # E > 1024
     assert call(f, 16, 2, 8, 0, f, f, f, None, None, 0, None) == lib.CHORD_ERR_UNSUPPORTED      # block_m = 0
     assert call(f, 16384, 8, 48, 8, f, f, f, None, None, 0, None) == lib.CHORD_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_wait_selftest_rejects_bad_args_before_touching_the_device(lib):
+    f = ctypes.c_void_p(0x100000)
+    call = _raw(lib).chord_selftest_wait_timeout
+    assert call(None, f, 1000, None) == lib.CHORD_ERR_INVALID_ARG
+    assert call(f, None, 1000, None) == lib.CHORD_ERR_INVALID_ARG
+    assert call(f, f, 0, None) == lib.CHORD_ERR_INVALID_ARG          # limit below 1 us
+    assert call(f, f, 1000001, None) == lib.CHORD_ERR_INVALID_ARG    # limit above 1 s
+    assert "limit_us" in lib.chord_last_error_detail()
+
+
+def test_align_workspace_follows_run_size(lib):
+    # multi-CTA routing sort: 256-slot runs while E x runs stays within 2^17 histogram
+    # entries, else 1024-slot runs (so the no-allocation variant's static scratch of
+    # 576 KiB always suffices up to 2^17 slots)
+    def runs_bytes(n, E, run):
+        g = -(-n // run)
+        a = lambda x: (x + 255) // 256 * 256
+        return a(E * g * 4) + a(E * 4) + a((E + 1) * 4)
+    assert lib.chord_moe_align_workspace_bytes(8192, 8, 48) == runs_bytes(8192 * 8, 48, 256)
+    assert lib.chord_moe_align_workspace_bytes(16384, 8, 1024) == runs_bytes(16384 * 8, 1024, 1024)
+    assert lib.chord_moe_align_workspace_bytes(16384, 8, 1024) <= 576 * 1024
