@@ -174,6 +174,58 @@ def recorded_traffic(kernel_key: str, workload: str):
     return rec["dram_bytes_per_launch"]
 
 
+def pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world):
+    """Device time of K end-to-end steps: every step copies its inputs in from pinned host
+    memory, runs the layer through the public API and copies the result back. Two buffer
+    slots: step k + 1's copy in (one stream) and step k - 1's copy out (another) overlap
+    step k's compute, as a serving loop runs them (PCIe is full duplex). Events order
+    each slot's reuse: inputs are rewritten only after the compute that read them, outputs
+    only after their copy out. The timed region runs from an event that both copy streams
+    wait on to one recorded after the last copy out."""
+    import torch
+
+    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_read = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for k in range(n):
+            s = k % 2
+            if k >= 2:
+                h2d.wait_event(done[s])
+            with torch.cuda.stream(h2d):
+                copy_in(s)
+            in_ready[s].record(h2d)
+            stream.wait_event(in_ready[s])
+            if k >= 2:
+                stream.wait_event(out_read[s])
+            with torch.cuda.stream(stream):
+                compute(s)
+            done[s].record(stream)
+            d2h.wait_event(done[s])
+            with torch.cuda.stream(d2h):
+                copy_out(s)
+            out_read[s].record(d2h)
+
+    run(W)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    last = torch.cuda.Event()
+    start.record(stream)
+    h2d.wait_event(start)
+    d2h.wait_event(start)
+    run(K)
+    last.record(d2h)
+    stream.wait_event(last)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(stop)
+
+
 def run_chord(args, rank, world, local_rank):
     import torch
     from w4a16_int4_mixture_align_b200 import chord
@@ -265,35 +317,31 @@ def run_chord(args, rank, world, local_rank):
     x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
     ids_h = torch.from_numpy(ids_np).pin_memory()
     tw_h = torch.from_numpy(tw_np).pin_memory()
-    out_h = torch.empty((cfg.T, cfg.H), dtype=torch.int16).pin_memory()
-    xd, idsd, twd = torch.empty_like(x), torch.empty_like(ids), torch.empty_like(tw)
+    out_h = [torch.empty((cfg.T, cfg.H), dtype=torch.int16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    idsd = [torch.empty_like(ids) for _ in range(2)]
+    twd = [torch.empty_like(tw) for _ in range(2)]
+    outd = [torch.empty_like(out) for _ in range(2)]
 
-    def e2e_step():
-        xd.view(torch.int16).copy_(x_h, non_blocking=True)
-        idsd.copy_(ids_h, non_blocking=True)
-        twd.copy_(tw_h, non_blocking=True)
-        layer.forward(xd, idsd, twd, out=out)
-        out_h.copy_(out.view(torch.int16), non_blocking=True)
+    def copy_in(s):
+        xd[s].view(torch.int16).copy_(x_h, non_blocking=True)
+        idsd[s].copy_(ids_h, non_blocking=True)
+        twd[s].copy_(tw_h, non_blocking=True)
 
-    for _ in range(W):
-        e2e_step()
-    barrier(world)
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e2.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
+    def compute(s):
+        layer.forward(xd[s], idsd[s], twd[s], out=outd[s])
+
+    def copy_out(s):
+        out_h[s].copy_(outd[s].view(torch.int16), non_blocking=True)
+
+    e2e_ms = pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world)
     sampler.stop()
-    e2e_ms = s2.elapsed_time(e2)
 
     # ---- the fused router + routing sort at this workload's shape (outside the timed
     # regions above; graph-replayed, so host marshalling does not hide device time)
     router_us = time_router(chord, cfg, rcfg, dev)
     h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
-    d2h = out_h.numel() * 2
+    d2h = out_h[0].numel() * 2
 
     # ---- max over ranks (outside the timed regions)
     stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
@@ -489,28 +537,23 @@ def run_grouped(args, rank, world, local_rank):
     # end to end: activations and routing from pinned host memory, the result back
     x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
     r_h = torch.from_numpy(route_np).pin_memory()
-    out_h = torch.empty((M, cfg.N), dtype=torch.int16).pin_memory()
-    xd, rd = torch.empty_like(x), torch.empty_like(route)
+    out_h = [torch.empty((M, cfg.N), dtype=torch.int16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    rd = [torch.empty_like(route) for _ in range(2)]
+    outd = [torch.empty_like(out) for _ in range(2)]
 
-    def e2e_step():
-        xd.view(torch.int16).copy_(x_h, non_blocking=True)
-        rd.copy_(r_h, non_blocking=True)
-        call(xd, rd, out)
-        out_h.copy_(out.view(torch.int16), non_blocking=True)
+    def copy_in(s):
+        xd[s].view(torch.int16).copy_(x_h, non_blocking=True)
+        rd[s].copy_(r_h, non_blocking=True)
 
-    for _ in range(W):
-        e2e_step()
-    barrier(world)
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e2.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
+    def compute(s):
+        call(xd[s], rd[s], outd[s])
+
+    def copy_out(s):
+        out_h[s].copy_(outd[s].view(torch.int16), non_blocking=True)
+
+    e2e_ms = pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world)
     sampler.stop()
-    e2e_ms = s2.elapsed_time(e2)
     stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
     elapsed_ms, e2e_ms, seg_ms = stats[0], stats[1], np.array(stats[2:])
     if rank != 0:
@@ -550,7 +593,7 @@ def run_grouped(args, rank, world, local_rank):
         "kernels_us": {"routing": round(seg_ms[0] * 1000, 2), "gemm": round(gemm_us, 2)},
         "roofline": roofline,
         "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
-                "h2d_bytes_per_step": x_h.numel() * 2 + r_h.numel() * 4, "d2h_bytes_per_step": out_h.numel() * 2},
+                "h2d_bytes_per_step": x_h.numel() * 2 + r_h.numel() * 4, "d2h_bytes_per_step": out_h[0].numel() * 2},
         "gpu_launches": int(launches),
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
