@@ -59,27 +59,45 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     for (int u = 0; u < kCombineVecs; ++u)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-    for (int j = 0; j < topk; ++j) {
-      const int64_t rj = __shfl_sync(0xffffffffu, j < 32 ? row[0] : row[1], j & 31);
-      const float wj = __shfl_sync(0xffffffffu, j < 32 ? w[0] : w[1], j & 31);
-      if (rj < 0) continue;
-      float4 v[kCombineVecs][2];
+    // slots in groups of kSlotGroup: the group's rows are all requested before any is
+    // summed (one memory round trip per group, not per slot), then added in ascending j
+    constexpr int kSlotGroup = 4;
+    for (int j0 = 0; j0 < topk; j0 += kSlotGroup) {
+      int64_t rj[kSlotGroup];
+      float wj[kSlotGroup];
+      float4 v[kSlotGroup][kCombineVecs][2];
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u) {
-        const int c = c0 + u * kCombineThreads * 8;
-        v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c < H) {
-          const float* src = BLOCKED ? y + ((int64_t(c >> 7) * cap + rj) << 7) + (c & 127) : y + rj * H + c;
-          v[u][0] = __ldcs(reinterpret_cast<const float4*>(src));
-          v[u][1] = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+      for (int q = 0; q < kSlotGroup; ++q) {
+        const int j = j0 + q;
+        rj[q] = -1;
+        wj[q] = 0.f;
+        if (j < topk) {
+          rj[q] = __shfl_sync(0xffffffffu, j < 32 ? row[0] : row[1], j & 31);
+          wj[q] = __shfl_sync(0xffffffffu, j < 32 ? w[0] : w[1], j & 31);
+        }
+#pragma unroll
+        for (int u = 0; u < kCombineVecs; ++u) {
+          const int c = c0 + u * kCombineThreads * 8;
+          v[q][u][0] = v[q][u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (rj[q] >= 0 && c < H) {
+            const float* src =
+                BLOCKED ? y + ((int64_t(c >> 7) * cap + rj[q]) << 7) + (c & 127) : y + rj[q] * H + c;
+            v[q][u][0] = __ldcs(reinterpret_cast<const float4*>(src));
+            v[q][u][1] = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+          }
         }
       }
       // product rounded, then added (no fused multiply-add), as the layer is defined
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u) {
-        const float vv[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+      for (int q = 0; q < kSlotGroup; ++q) {
+        if (rj[q] < 0) continue;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(wj, vv[i]));
+        for (int u = 0; u < kCombineVecs; ++u) {
+          const float vv[8] = {v[q][u][0].x, v[q][u][0].y, v[q][u][0].z, v[q][u][0].w,
+                               v[q][u][1].x, v[q][u][1].y, v[q][u][1].z, v[q][u][1].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(wj[q], vv[i]));
+        }
       }
     }
 #pragma unroll
