@@ -284,6 +284,10 @@ CHORD_API chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t 
  * [0] right before their GEMM kernel and [1] after it. Records use cudaEventRecordExternal,
  * so a forward captured into a CUDA graph records them when the graph is replayed. n == 0 clears the hook. The handles must stay
  * valid while set. Returns CHORD_ERR_INVALID_ARG for other n or null handles.
+ * Without the hook, the layer's GEMM and combine kernels on the weight-streaming schedule
+ * are launched early (programmatic dependent launch: each waits on the device for the
+ * previous kernel's output); an event between two kernels orders them fully, so while the
+ * hook is set they are launched plainly.
  *
  * chord_launch_count: number of CUDA kernels this library has launched in the process
  * (all entry points, all threads), for checking launch counts of a timed region.
