@@ -259,6 +259,43 @@ def test_forward_ep_shard_with_nonlocal_slots():
     assert np.abs(f32(got) - ref).max() <= 8e-3 * np.abs(ref).max()
 
 
+def test_ep_shards_add_up_to_the_unsharded_layer():
+    """Expert parallelism splits the experts over shards and each shard keeps the global
+    top-k weights (not renormalised over its local experts), so the shard outputs add up
+    to the unsharded layer, up to one bf16 rounding per shard. Renormalising the weights
+    per shard, or dropping slots that carry another shard's global id, would break this."""
+    E_all, shards, topk = 12, 3, 3
+    d = tiny_inputs(seed=7, T=24, E=E_all, topk=topk)
+    full = f32(run_oracle(d))
+    per = E_all // shards
+    total = np.zeros_like(full)
+    for r in range(shards):
+        lo = r * per
+        ids = d["topk_ids"].copy()
+        local = (ids >= lo) & (ids < lo + per)
+        # local slots renumbered to this shard's experts; the others keep a global id
+        # at or past the shard's E, which marks a slot of another shard
+        ids = np.where(local, ids - lo, ids + per)
+        shard = dict(d, topk_ids=ids.astype(np.int32),
+                     qw13=np.ascontiguousarray(d["qw13"][lo:lo + per]), s13=np.ascontiguousarray(d["s13"][lo:lo + per]),
+                     qw2=np.ascontiguousarray(d["qw2"][lo:lo + per]), s2=np.ascontiguousarray(d["s2"][lo:lo + per]))
+        total += f32(run_oracle(shard))
+    assert np.abs(total - full).max() <= 4 * 2.0 ** -8 * np.abs(full).max()
+    # renormalising the weights over each shard's local slots does not add up
+    wrong = np.zeros_like(full)
+    for r in range(shards):
+        lo = r * per
+        local = (d["topk_ids"] >= lo) & (d["topk_ids"] < lo + per)
+        w = np.where(local, d["topk_weights"], 0.0)
+        w = (w / np.maximum(w.sum(axis=1, keepdims=True), 1e-30)).astype(np.float32)
+        ids = np.where(local, d["topk_ids"] - lo, -1).astype(np.int32)
+        shard = dict(d, topk_ids=ids, topk_weights=w,
+                     qw13=np.ascontiguousarray(d["qw13"][lo:lo + per]), s13=np.ascontiguousarray(d["s13"][lo:lo + per]),
+                     qw2=np.ascontiguousarray(d["qw2"][lo:lo + per]), s2=np.ascontiguousarray(d["s2"][lo:lo + per]))
+        wrong += f32(run_oracle(shard))
+    assert np.abs(wrong - full).max() > 0.1 * np.abs(full).max()
+
+
 def test_subset_rows_equal_full_rows():
     d = tiny_inputs(seed=3)
     full = run_oracle(d)
