@@ -414,7 +414,7 @@ def time_router(chord, cfg, rcfg, dev, calls=20, replays=10):
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     s = torch.empty(chord.chord_moe_align_capacity(T, k, E, bm), dtype=torch.int32, device=dev)
     e = torch.empty(max(chord.chord_moe_align_num_blocks(T, k, E, bm), 1), dtype=torch.int32, device=dev)
-    n = torch.empty(1, dtype=torch.int32, device=dev)
+    n = torch.empty(2, dtype=torch.int32, device=dev)  # padded count, routing tag
     wsb = chord.chord_moe_align_workspace_bytes(T, k, E)
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev) if wsb else None
     side = torch.cuda.Stream(device=dev)

@@ -64,6 +64,13 @@ typedef enum {
 #define CHORD_DEV_ROUTING_INVALID 0x1u /* VALIDATE_ROUTING found inconsistent routing */
 #define CHORD_DEV_BLOB_MISMATCH   0x2u /* a weight blob header does not match the call */
 #define CHORD_DEV_TIMEOUT         0x4u /* a bounded on-chip wait gave up */
+#define CHORD_DEV_BLOCK_M_MISMATCH 0x8u /* routing tensors built for another block_m: nothing computed */
+
+/* The routing tag: word [1] of num_tokens_padded, written by every routing entry point
+ * (chord_moe_align, chord_moe_align_noalloc, chord_router_topk_align) and checked on the
+ * device by chord_moe_forward before it reads expert_ids. A producer of routing tensors
+ * other than this library must write it too. */
+#define CHORD_ROUTING_TAG(block_m) ((int32_t)(0x52540000u | (uint32_t)(block_m)))
 
 /* Weight roles for chord_repack_weights. */
 #define CHORD_ROLE_GATE_UP 1 /* W13 [E, 2I, H]: rows [0,I) gate, rows [I,2I) up */
@@ -92,6 +99,9 @@ CHORD_API const char* chord_last_error_detail(void);
  *   expert_ids[b] = e for the p_e / block_m blocks of expert e, in increasing e, and
  *   -1 for every block at or past num_tokens_padded / block_m;
  *   num_tokens_padded[0] = off_E;   expert_offsets[e] = off_e for e in [0, E].
+ *   num_tokens_padded[1] = CHORD_ROUTING_TAG(block_m): the block_m these tensors were
+ *   built for, which chord_moe_forward checks on the device (the padded count alone does
+ *   not reveal it, and a forward with another block_m would misread expert_ids).
  * An expert with no local slot gets no block. The result is deterministic.
  *
  * Capacities: sorted_ids holds chord_moe_align_capacity() int32, expert_ids holds
@@ -105,7 +115,7 @@ CHORD_API int64_t chord_moe_align_num_blocks(int64_t T, int topk, int E, int blo
 CHORD_API size_t chord_moe_align_workspace_bytes(int64_t T, int topk, int E);
 CHORD_API chord_status_t chord_moe_align(const int32_t* topk_ids /* device [T, topk] */, int64_t T,
                                int topk, int E, int block_m, int32_t* sorted_ids,
-                               int32_t* expert_ids, int32_t* num_tokens_padded /* [1] */,
+                               int32_t* expert_ids, int32_t* num_tokens_padded /* [2] */,
                                int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
                                size_t workspace_bytes, chord_stream_t stream);
 
@@ -133,7 +143,7 @@ CHORD_API chord_status_t chord_moe_align(const int32_t* topk_ids /* device [T, t
 CHORD_API chord_status_t chord_router_topk_align(const float* logits, int64_t T, int E_global, int topk, int E,
                                                  int block_m, int32_t* topk_ids, float* topk_weights,
                                                  int32_t* sorted_ids, int32_t* expert_ids,
-                                                 int32_t* num_tokens_padded /* [1] */,
+                                                 int32_t* num_tokens_padded /* [2] */,
                                                  int32_t* expert_offsets /* [E+1] or NULL */, void* workspace,
                                                  size_t workspace_bytes, chord_stream_t stream);
 
@@ -151,8 +161,9 @@ CHORD_API chord_status_t chord_router_topk_align(const float* logits, int64_t T,
  *  - All calls share the array. Nothing in it needs to start at zero (each call
  *    overwrites every entry it later reads), but calls that overlap on the GPU (other
  *    streams, other host threads) race on it: serialise them.
- * Returns CHORD_ERR_INVALID_ARG for bad sizes or null pointers, CHORD_ERR_CUDA when the
- * address lookup or a launch fails. */
+ * Returns the status chord_moe_align returns for the same arguments (with the same
+ * chord_last_error_detail() text), plus CHORD_ERR_UNSUPPORTED with a detail naming the
+ * limit when T*topk exceeds 2^17, and CHORD_ERR_CUDA when the address lookup fails. */
 CHORD_API chord_status_t chord_moe_align_noalloc(const int32_t* topk_ids, int64_t T, int topk, int E,
                                                  int block_m, int32_t* sorted_ids, int32_t* expert_ids,
                                                  int32_t* num_tokens_padded, int32_t* expert_offsets,
@@ -203,7 +214,11 @@ CHORD_API int chord_select_block_m(int64_t T, int topk, int E_local, int E_globa
  * topk_weights device fp32  [T, topk]; not renormalised over local slots
  * sorted_ids, expert_ids, num_tokens_padded: device routing tensors for this block_m
  *              (from chord_moe_align or any producer with the same contract; entries
- *              >= T*topk are padding, blocks with expert_ids outside [0,E) are skipped)
+ *              >= T*topk are padding, blocks with expert_ids outside [0,E) are skipped).
+ *              num_tokens_padded[1] must be CHORD_ROUTING_TAG(block_m); otherwise the
+ *              kernels read no other routing tensor, compute nothing, write zero rows
+ *              to `out` and set CHORD_DEV_BLOCK_M_MISMATCH (checked on the device, so a
+ *              captured graph needs no readback).
  * w13, w2      device blobs from chord_repack_weights (roles GATE_UP [E,2I,H], DOWN [E,H,I])
  * out          device bf16 [T, H]; every row is written (0 for tokens with no local slot)
  * workspace    device, >= chord_moe_workspace_bytes(), 256-byte aligned. Its first 256

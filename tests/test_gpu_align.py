@@ -28,12 +28,13 @@ def run_align(chord, ids: np.ndarray, E: int, bm: int):
     # poison outputs so unwritten entries are caught
     s = torch.full((max(cap, 1),), -7, dtype=torch.int32, device=dev)
     e = torch.full((max(nb, 1),), -7, dtype=torch.int32, device=dev)
-    n = torch.full((1,), -7, dtype=torch.int32, device=dev)
+    n = torch.full((2,), -7, dtype=torch.int32, device=dev)
     o = torch.full((E + 1,), -7, dtype=torch.int32, device=dev)
     wsb = chord.chord_moe_align_workspace_bytes(T, k, E)
     ws = torch.full((max(wsb, 1),), 0x5A, dtype=torch.uint8, device=dev) if wsb else None
     chord.chord_moe_align(d_ids, E, bm, s, e, n, o, ws)
     torch.cuda.synchronize()
+    assert int(n.cpu()[1]) == chord.routing_tag(bm)  # the block_m the forward checks
     return s.cpu().numpy()[:cap], e.cpu().numpy()[:nb], int(n.cpu()[0]), o.cpu().numpy()
 
 

@@ -219,3 +219,25 @@ def test_routing_validation_flags_corrupt_tensors(chord, tiny):
                             layer.block_m, layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace,
                             chord.CHORD_FLAG_VALIDATE_ROUTING)
     assert layer.check_status() == 0
+
+
+@pytest.mark.parametrize("path", ["stream", "tensor"])
+@pytest.mark.parametrize("bm_align,bm_forward", [(16, 8), (8, 16), (8, 64), (64, 8)])
+def test_block_m_mismatch_is_caught_on_the_device(chord, tiny, path, bm_align, bm_forward):
+    # routing sorted for one block_m, forward called with another: the kernels check the
+    # tag in num_tokens_padded[1] before reading expert_ids, compute nothing, write zero
+    # rows and raise CHORD_DEV_BLOCK_M_MISMATCH (no host readback)
+    import torch
+    src = make_layer(chord, tiny, block_m=bm_align)
+    dst = make_layer(chord, tiny, block_m=bm_forward)  # workspace sized for bm_forward
+    t = to_dev(tiny)
+    src.align(t["ids"])
+    flags = chord.CHORD_FLAG_FORCE_STREAM if path == "stream" else chord.CHORD_FLAG_FORCE_TENSOR
+    out = torch.full((16, 256), 1.0, dtype=torch.bfloat16, device="cuda")
+    chord.chord_moe_forward(t["x"], t["ids"], t["w"], src.sorted_ids, src.expert_ids, src.ntp, bm_forward,
+                            dst.w13, dst.w2, dst.I, dst.E, out, dst.workspace, flags)
+    assert dst.check_status() == chord.CHORD_DEV_BLOCK_M_MISMATCH
+    assert torch.count_nonzero(out.float()).item() == 0
+    # the matching block_m on the same buffers still computes the layer
+    got = run_layer(dst, tiny, flags)
+    assert_layer_close(got, oracle_rows(tiny, None))

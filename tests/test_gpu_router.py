@@ -44,12 +44,13 @@ def run_router(chord, logits, topk, E, bm):
     w = torch.full((T, topk), -7.0, dtype=torch.float32, device=dev)
     s = torch.full((max(cap, 1),), -7, dtype=torch.int32, device=dev)
     e = torch.full((max(nb, 1),), -7, dtype=torch.int32, device=dev)
-    n = torch.full((1,), -7, dtype=torch.int32, device=dev)
+    n = torch.full((2,), -7, dtype=torch.int32, device=dev)
     o = torch.full((E + 1,), -7, dtype=torch.int32, device=dev)
     wsb = chord.chord_moe_align_workspace_bytes(T, topk, E)
     ws = torch.full((max(wsb, 1),), 0x5A, dtype=torch.uint8, device=dev) if wsb else None
     chord.chord_router_topk_align(lg, topk, E, bm, ids, w, s, e, n, o, ws)
     torch.cuda.synchronize()
+    assert int(n.cpu()[1]) == chord.routing_tag(bm)
     return (ids.cpu().numpy(), w.cpu().numpy(), s.cpu().numpy()[:cap], e.cpu().numpy()[:nb],
             int(n.cpu()[0]), o.cpu().numpy())
 

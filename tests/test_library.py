@@ -130,3 +130,31 @@ def test_align_workspace_follows_run_size(lib):
     assert lib.chord_moe_align_workspace_bytes(8192, 8, 48) == runs_bytes(8192 * 8, 48, 256)
     assert lib.chord_moe_align_workspace_bytes(16384, 8, 1024) == runs_bytes(16384 * 8, 1024, 1024)
     assert lib.chord_moe_align_workspace_bytes(16384, 8, 1024) <= 576 * 1024
+
+
+def test_noalloc_reports_what_chord_moe_align_reports(lib):
+    # the no-allocation routing sort shares chord_moe_align's checks, statuses and detail
+    # texts; these fail before any device access
+    f = ctypes.c_void_p(0x100000)
+    ws = _raw(lib).chord_moe_align
+    na = _raw(lib).chord_moe_align_noalloc
+    cases = [(16, 2, 0, 8), (16, 2, 2000, 8), (16, 2, 8, 0), (16, 2, 8, 300), (-1, 2, 8, 8), (16, 0, 8, 8),
+             (1 << 62, 8, 48, 8), (1 << 28, 8, 48, 8)]
+    for T, k, E, bm in cases:
+        a = ws(f, T, k, E, bm, f, f, f, None, f, 1 << 40, None)
+        da = lib.chord_last_error_detail()
+        b = na(f, T, k, E, bm, f, f, f, None, None)
+        db = lib.chord_last_error_detail()
+        assert a == b != lib.CHORD_OK and da == db, (T, k, E, bm, a, b, da, db)
+    assert na(None, 16, 2, 8, 8, f, f, f, None, None) == lib.CHORD_ERR_INVALID_ARG  # null ids
+    assert "null" in lib.chord_last_error_detail()
+    # its own limit: the static scratch holds the histograms of up to 2^17 slots
+    assert na(f, 16385, 8, 48, 16, f, f, f, None, None) == lib.CHORD_ERR_UNSUPPORTED
+    assert "static scratch" in lib.chord_last_error_detail()
+
+
+def test_align_size_checks_do_not_overflow(lib):
+    # T * topk is bounded before it is formed: T near 2^62 must be refused, not wrap
+    f = ctypes.c_void_p(0x100000)
+    st = _raw(lib).chord_moe_align(f, (1 << 62) + 1, 64, 48, 8, f, f, f, None, f, 1 << 40, None)
+    assert st == lib.CHORD_ERR_UNSUPPORTED and "2^31" in lib.chord_last_error_detail()

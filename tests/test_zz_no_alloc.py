@@ -26,7 +26,7 @@ def _buffers(chord, T, k, E, bm):
     cap = chord.chord_moe_align_capacity(T, k, E, bm)
     nb = chord.chord_moe_align_num_blocks(T, k, E, bm)
     mk = lambda n: torch.full((max(n, 1),), -7, dtype=torch.int32, device="cuda")  # noqa: E731
-    return mk(cap), mk(nb), mk(1), mk(E + 1), cap, nb
+    return mk(cap), mk(nb), mk(2), mk(E + 1), cap, nb
 
 
 def _with_workspace(chord, ids, E, bm):
@@ -37,7 +37,7 @@ def _with_workspace(chord, ids, E, bm):
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda") if wsb else None
     chord.chord_moe_align(ids, E, bm, s, e, n, o, ws)
     torch.cuda.synchronize()
-    return [t.cpu().numpy()[:m] for t, m in ((s, cap), (e, nb), (n, 1), (o, E + 1))]
+    return [t.cpu().numpy()[:m] for t, m in ((s, cap), (e, nb), (n, 2), (o, E + 1))]
 
 
 def _noalloc(chord, ids, E, bm):
@@ -46,7 +46,7 @@ def _noalloc(chord, ids, E, bm):
     s, e, n, o, cap, nb = _buffers(chord, T, k, E, bm)
     chord.chord_moe_align_noalloc(ids, E, bm, s, e, n, o)
     torch.cuda.synchronize()
-    return [t.cpu().numpy()[:m] for t, m in ((s, cap), (e, nb), (n, 1), (o, E + 1))]
+    return [t.cpu().numpy()[:m] for t, m in ((s, cap), (e, nb), (n, 2), (o, E + 1))]
 
 
 @pytest.mark.parametrize("name,bm", [("ep8_decode", 8), ("skew", 256), ("ep8_prefill", 16), ("tp8_prefill", 64)])
@@ -77,3 +77,4 @@ def test_noalloc_refuses_batches_past_the_static_limit(chord):
     with pytest.raises(chord.ChordError) as ei:
         chord.chord_moe_align_noalloc(ids, 48, 16, s, e, n, o)
     assert ei.value.status == chord.CHORD_ERR_UNSUPPORTED
+    assert "static scratch" in chord.chord_last_error_detail()

@@ -25,6 +25,13 @@ CHORD_ERR_DEVICE = 6
 CHORD_DEV_ROUTING_INVALID = 0x1
 CHORD_DEV_BLOB_MISMATCH = 0x2
 CHORD_DEV_TIMEOUT = 0x4
+CHORD_DEV_BLOCK_M_MISMATCH = 0x8
+
+
+def routing_tag(block_m: int) -> int:
+    """num_tokens_padded[1] as the routing entry points write it (CHORD_ROUTING_TAG)."""
+    v = 0x52540000 | int(block_m)
+    return v - (1 << 32) if v >= 1 << 31 else v
 
 CHORD_ROLE_GATE_UP = 1
 CHORD_ROLE_DOWN = 2
@@ -111,6 +118,12 @@ def _nbytes(t) -> int:
     return t.numel() * t.element_size()
 
 
+def _routing_header(t):
+    # num_tokens_padded holds two int32: the padded count and the routing tag
+    assert t.dtype == torch.int32 and t.numel() >= 2, "num_tokens_padded must be an int32 tensor of 2 elements"
+    return t
+
+
 # --------------------------------------------------------------------------- sizes
 
 def chord_moe_align_capacity(T, topk, E, block_m) -> int:
@@ -152,7 +165,7 @@ def chord_moe_align(topk_ids, E, block_m, sorted_ids, expert_ids, num_tokens_pad
     T, topk = topk_ids.shape
     ws_bytes = 0 if workspace is None else _nbytes(workspace)
     _check(lib().chord_moe_align(_ptr(topk_ids), T, topk, E, block_m, _ptr(sorted_ids),
-                                 _ptr(expert_ids), _ptr(num_tokens_padded), _ptr(expert_offsets),
+                                 _ptr(expert_ids), _ptr(_routing_header(num_tokens_padded)), _ptr(expert_offsets),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "chord_moe_align")
 
 
@@ -162,7 +175,7 @@ def chord_moe_align_noalloc(topk_ids, E, block_m, sorted_ids, expert_ids, num_to
     library (for callers that cannot allocate device memory when they route)."""
     T, topk = topk_ids.shape
     _check(lib().chord_moe_align_noalloc(_ptr(topk_ids), T, topk, E, block_m, _ptr(sorted_ids),
-                                         _ptr(expert_ids), _ptr(num_tokens_padded),
+                                         _ptr(expert_ids), _ptr(_routing_header(num_tokens_padded)),
                                          _ptr(expert_offsets), _stream(stream)),
            "chord_moe_align_noalloc")
 
@@ -175,7 +188,7 @@ def chord_router_topk_align(logits, topk, E, block_m, topk_ids, topk_weights, so
     ws_bytes = 0 if workspace is None else _nbytes(workspace)
     _check(lib().chord_router_topk_align(_ptr(logits), T, E_global, topk, E, block_m, _ptr(topk_ids),
                                          _ptr(topk_weights), _ptr(sorted_ids), _ptr(expert_ids),
-                                         _ptr(num_tokens_padded), _ptr(expert_offsets), _ptr(workspace),
+                                         _ptr(_routing_header(num_tokens_padded)), _ptr(expert_offsets), _ptr(workspace),
                                          ws_bytes, _stream(stream)), "chord_router_topk_align")
 
 
@@ -196,7 +209,7 @@ def chord_moe_forward(hidden, topk_ids, topk_weights, sorted_ids, expert_ids, nu
     T, H = hidden.shape
     topk = topk_ids.shape[1]
     _check(lib().chord_moe_forward(_ptr(hidden), _ptr(topk_ids), _ptr(topk_weights),
-                                   _ptr(sorted_ids), _ptr(expert_ids), _ptr(num_tokens_padded),
+                                   _ptr(sorted_ids), _ptr(expert_ids), _ptr(_routing_header(num_tokens_padded)),
                                    block_m, _ptr(w13), _ptr(w2), T, H, I, E, topk, _ptr(out),
                                    _ptr(workspace), _nbytes(workspace), flags, _stream(stream)),
            "chord_moe_forward")
@@ -292,7 +305,7 @@ class ChordMoE:
         d = self.device
         self.sorted_ids = torch.empty(max(cap, 1), dtype=torch.int32, device=d)
         self.expert_ids = torch.empty(max(nb, 1), dtype=torch.int32, device=d)
-        self.ntp = torch.zeros(1, dtype=torch.int32, device=d)
+        self.ntp = torch.zeros(2, dtype=torch.int32, device=d)  # padded count, routing tag
         self.offsets = torch.empty(self.E + 1, dtype=torch.int32, device=d)
         aw = chord_moe_align_workspace_bytes(T, self.topk, self.E)
         self.align_ws = _alloc_bytes(aw, d) if aw else None

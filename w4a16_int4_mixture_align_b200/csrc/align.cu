@@ -212,7 +212,10 @@ __device__ __forceinline__ void align_single_body(
 
   if (c0 < n) chunk_scatter(v, steps, c0, E, nbits, hist + warp * E, sorted_ids);
   fill_tail(cnt, off, E, block_m, n, cap, nblocks, sorted_ids, expert_ids, tid, blockDim.x);
-  if (tid == 0) *ntp_out = off[E];
+  if (tid == 0) {
+    ntp_out[0] = off[E];
+    ntp_out[1] = routing_tag(block_m);
+  }
   if (offsets_out)
     for (int e = tid; e <= E; e += blockDim.x) offsets_out[e] = off[e];
 }
@@ -421,7 +424,8 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int E, int block_m, in
   for (int e = tid; e < E; e += blockDim.x) off_g[e] = off[e];
   if (tid == 0) {
     off_g[E] = total;
-    *ntp_out = total;
+    ntp_out[0] = total;
+    ntp_out[1] = routing_tag(block_m);
   }
   if (offsets_out) {
     for (int e = tid; e < E; e += blockDim.x) offsets_out[e] = off[e];

@@ -54,23 +54,24 @@ extern "C" chord_status_t chord_moe_align_noalloc(const int32_t* topk_ids, int64
                                                   int block_m, int32_t* sorted_ids, int32_t* expert_ids,
                                                   int32_t* num_tokens_padded, int32_t* expert_offsets,
                                                   chord_stream_t stream) {
-  if (T < 0 || topk < 1 || topk > 64 || E < 1 || E > 1024 || block_m < 1 || block_m > 256)
-    return CHORD_ERR_INVALID_ARG;
-  if (T * topk > kStaticMaxSlots) return CHORD_ERR_UNSUPPORTED;  // beyond the static scratch
+  // the same checks, statuses and detail texts as chord_moe_align, in the same order
+  clear_detail();
+  chord_status_t st = check_align_args(T, topk, E, block_m);
+  if (st != CHORD_OK) return st;
   if ((T > 0 && !topk_ids) || !sorted_ids || !expert_ids || !num_tokens_padded)
-    return CHORD_ERR_INVALID_ARG;
+    return fail(CHORD_ERR_INVALID_ARG, "null routing pointer");
+  // the one limit of its own: the static scratch (T*topk < 2^31 is already checked)
+  if (T * topk > kStaticMaxSlots || align_workspace_bytes(T * topk, E) > kStaticScratchBytes)
+    return fail(CHORD_ERR_UNSUPPORTED, "T*topk=%lld exceeds the static scratch limit of %lld slots",
+                (long long)(T * topk), (long long)kStaticMaxSlots);
+  if ((st = current_device(nullptr)) != CHORD_OK) return st;
+  void* scratch = nullptr;
+  cudaError_t err = scratch_address(&scratch);
+  if (err != cudaSuccess) return cuda_fail(err, "static scratch address (cudaGetSymbolAddress)");
   const int64_t cap = T * topk + int64_t(E) * (block_m - 1);
   const int64_t nblocks = (cap + block_m - 1) / block_m;
-  if (align_workspace_bytes(T * topk, E) > kStaticScratchBytes) return CHORD_ERR_UNSUPPORTED;
-  void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return CHORD_ERR_CUDA;
-  int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CHORD_ERR_CUDA;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (major != 10 || minor != 0) return CHORD_ERR_UNSUPPORTED;
-  const cudaError_t err = launch_align(topk_ids, T * topk, E, block_m, cap, nblocks, sorted_ids, expert_ids,
-                                       num_tokens_padded, expert_offsets, scratch,
-                                       reinterpret_cast<cudaStream_t>(stream));
-  return err == cudaSuccess ? CHORD_OK : CHORD_ERR_CUDA;
+  err = launch_align(topk_ids, T * topk, E, block_m, cap, nblocks, sorted_ids, expert_ids, num_tokens_padded,
+                     expert_offsets, scratch, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_align launch");
+  return CHORD_OK;
 }

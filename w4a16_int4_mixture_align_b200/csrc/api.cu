@@ -18,18 +18,6 @@ thread_local cudaEvent_t g_timing[4] = {nullptr, nullptr, nullptr, nullptr};
 thread_local bool g_timing_on = false;
 std::atomic<uint64_t> g_launches{0};
 
-chord_status_t fail(chord_status_t st, const char* fmt, ...) {
-  va_list ap;
-  va_start(ap, fmt);
-  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
-  va_end(ap);
-  return st;
-}
-
-chord_status_t cuda_fail(cudaError_t err, const char* what) {
-  return fail(CHORD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
-}
-
 struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
@@ -46,28 +34,48 @@ struct BlobInfo {
 std::unordered_map<const void*, BlobInfo> g_blobs;
 std::map<std::tuple<int64_t, int, int, int, int, int>, int> g_select_cache;
 
-chord_status_t current_device(DeviceInfo* out) {
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+}  // namespace
+
+chord_status_t fail(chord_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+chord_status_t cuda_fail(cudaError_t err, const char* what) {
+  return fail(CHORD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+void clear_detail() { g_detail[0] = 0; }
+
+chord_status_t current_device(int* num_sms) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
-  std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_devices.find(dev);
-  if (it == g_devices.end()) {
-    DeviceInfo d;
-    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-    d.ok = (d.major == 10 && d.minor == 0);
-    it = g_devices.emplace(dev, d).first;
+  DeviceInfo d;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_devices.find(dev);
+    if (it == g_devices.end()) {
+      DeviceInfo nd;
+      cudaDeviceGetAttribute(&nd.major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&nd.minor, cudaDevAttrComputeCapabilityMinor, dev);
+      cudaDeviceGetAttribute(&nd.num_sms, cudaDevAttrMultiProcessorCount, dev);
+      nd.ok = (nd.major == 10 && nd.minor == 0);
+      it = g_devices.emplace(dev, nd).first;
+    }
+    d = it->second;
   }
-  *out = it->second;
-  if (!out->ok)
-    return fail(CHORD_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
-                dev, out->major, out->minor);
+  if (num_sms) *num_sms = d.num_sms;
+  if (!d.ok)
+    return fail(CHORD_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, d.major,
+                d.minor);
   return CHORD_OK;
 }
-
-bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
 
 chord_status_t check_align_args(int64_t T, int topk, int E, int block_m) {
   if (T < 0 || topk < 1 || topk > 64)
@@ -75,12 +83,13 @@ chord_status_t check_align_args(int64_t T, int topk, int E, int block_m) {
   if (E < 1 || E > 1024) return fail(CHORD_ERR_UNSUPPORTED, "E=%d outside [1, 1024]", E);
   if (block_m < 1 || block_m > 256)
     return fail(CHORD_ERR_UNSUPPORTED, "block_m=%d outside [1, 256]", block_m);
+  // bounded before multiplying, so the product below cannot overflow
+  const int64_t lim = int64_t(1) << 31;
+  if (T >= lim / topk) return fail(CHORD_ERR_UNSUPPORTED, "T*topk (T=%lld, topk=%d) >= 2^31", (long long)T, topk);
   const int64_t cap = T * topk + int64_t(E) * (block_m - 1);
-  if (cap >= (int64_t(1) << 31)) return fail(CHORD_ERR_UNSUPPORTED, "routing capacity %lld >= 2^31", (long long)cap);
+  if (cap >= lim) return fail(CHORD_ERR_UNSUPPORTED, "routing capacity %lld >= 2^31", (long long)cap);
   return CHORD_OK;
 }
-
-}  // namespace
 
 void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
 
@@ -125,7 +134,7 @@ chord_status_t chord_moe_align(const int32_t* topk_ids, int64_t T, int topk, int
                                int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_tokens_padded,
                                int32_t* expert_offsets, void* workspace, size_t workspace_bytes,
                                chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   chord_status_t st = check_align_args(T, topk, E, block_m);
   if (st != CHORD_OK) return st;
   if ((T > 0 && !topk_ids) || !sorted_ids || !expert_ids || !num_tokens_padded)
@@ -135,8 +144,7 @@ chord_status_t chord_moe_align(const int32_t* topk_ids, int64_t T, int topk, int
     return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "align workspace needs %zu bytes, got %zu", need,
                 workspace ? workspace_bytes : size_t(0));
   if (need > 0 && !aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if ((st = current_device(nullptr)) != CHORD_OK) return st;
   const int64_t cap = chord_moe_align_capacity(T, topk, E, block_m);
   const int64_t nblocks = chord_moe_align_num_blocks(T, topk, E, block_m);
   cudaError_t err = launch_align(topk_ids, T * topk, E, block_m, cap, nblocks, sorted_ids,
@@ -150,7 +158,7 @@ chord_status_t chord_router_topk_align(const float* logits, int64_t T, int E_glo
                                        int block_m, int32_t* topk_ids, float* topk_weights, int32_t* sorted_ids,
                                        int32_t* expert_ids, int32_t* num_tokens_padded, int32_t* expert_offsets,
                                        void* workspace, size_t workspace_bytes, chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   chord_status_t st = check_align_args(T, topk, E, block_m);
   if (st != CHORD_OK) return st;
   if (E_global < topk || E_global > 1024)
@@ -162,8 +170,7 @@ chord_status_t chord_router_topk_align(const float* logits, int64_t T, int E_glo
     return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "align workspace needs %zu bytes, got %zu", need,
                 workspace ? workspace_bytes : size_t(0));
   if (need > 0 && !aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if ((st = current_device(nullptr)) != CHORD_OK) return st;
   const int64_t cap = chord_moe_align_capacity(T, topk, E, block_m);
   const int64_t nblocks = chord_moe_align_num_blocks(T, topk, E, block_m);
   cudaError_t err = launch_router_align(logits, T, E_global, topk, topk_ids, topk_weights, E, block_m, cap,
@@ -181,7 +188,7 @@ size_t chord_repacked_bytes(int E, int N, int K, int group_size) {
 chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scales, int E, int N,
                                     int K, int group_size, int role, void* out, size_t out_bytes,
                                     chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   if (group_size != kGroup)
     return fail(CHORD_ERR_UNSUPPORTED, "group_size=%d; only group-32 scales are supported", group_size);
   if (role < CHORD_ROLE_GATE_UP || role > CHORD_ROLE_GROUPED_MASKED)
@@ -194,8 +201,7 @@ chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scal
   const size_t need = size_t(blob_total_bytes(E, N, K));
   if (out_bytes < need) return fail(CHORD_ERR_INVALID_ARG, "blob needs %zu bytes, got %zu", need, out_bytes);
   chord_status_t st;
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if ((st = current_device(nullptr)) != CHORD_OK) return st;
   cudaError_t err = launch_repack(qweight, scales, E, N, K, role, static_cast<uint8_t*>(out),
                                   reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "repack launch");
@@ -206,7 +212,7 @@ chord_status_t chord_repack_weights(const int32_t* qweight, const uint16_t* scal
 
 chord_status_t chord_dequant_weights(const void* blob, size_t blob_bytes, uint16_t* w_bf16,
                                      chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   if (!blob || !w_bf16) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
   BlobInfo info;
   {
@@ -218,8 +224,7 @@ chord_status_t chord_dequant_weights(const void* blob, size_t blob_bytes, uint16
   }
   if (blob_bytes < info.bytes) return fail(CHORD_ERR_INVALID_ARG, "blob_bytes too small");
   chord_status_t st;
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  if ((st = current_device(nullptr)) != CHORD_OK) return st;
   cudaError_t err = launch_dequant_blob(static_cast<const uint8_t*>(blob), info.E, info.N, info.K,
                                         info.role, w_bf16, reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "dequant launch");
@@ -263,7 +268,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
                                  int block_m, const void* w13, const void* w2, int64_t T, int H,
                                  int I, int E, int topk, uint16_t* out, void* workspace,
                                  size_t workspace_bytes, int flags, chord_stream_t stream_) {
-  g_detail[0] = 0;
+  clear_detail();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   chord_status_t st = check_align_args(T, topk, E, block_m);
   if (st != CHORD_OK) return st;
@@ -297,8 +302,8 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
     if ((st = check(w13, CHORD_ROLE_GATE_UP, 2 * I, H, "w13")) != CHORD_OK) return st;
     if ((st = check(w2, CHORD_ROLE_DOWN, H, I, "w2")) != CHORD_OK) return st;
   }
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
   if (T == 0) return CHORD_OK;
 
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -324,7 +329,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   a.topk = topk;
   a.block_m = block_m;
   a.cap = chord_moe_align_capacity(T, topk, E, block_m);
-  a.num_sms = dev.num_sms;
+  a.num_sms = num_sms;
 
   cudaError_t err;
   if (flags & CHORD_FLAG_VALIDATE_ROUTING) {
@@ -390,8 +395,8 @@ chord_status_t grouped_gemm(const uint16_t* x, int64_t rows, int K, const int32_
     }
   }
   chord_status_t st;
-  DeviceInfo dev;
-  if ((st = current_device(&dev)) != CHORD_OK) return st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
   if (rows == 0) return CHORD_OK;
 
   // schedule: few rows per expert stream the weights (mma.sync over units of 8, 16 or 32
@@ -417,7 +422,7 @@ chord_status_t grouped_gemm(const uint16_t* x, int64_t rows, int K, const int32_
   g.bm = bm;
   g.cap = ws.max_positions;
   g.status = reinterpret_cast<uint32_t*>(wsb);
-  g.num_sms = dev.num_sms;
+  g.num_sms = num_sms;
   cudaError_t err = launch_grouped_route(m_indices, rows, masked_m, E, max_m, bm,
                                          const_cast<int32_t*>(g.expert_ids), const_cast<int32_t*>(g.block_row0),
                                          const_cast<int32_t*>(g.sorted_ids), const_cast<int32_t*>(g.ntp), g.status,
@@ -436,7 +441,7 @@ chord_status_t grouped_gemm(const uint16_t* x, int64_t rows, int K, const int32_
 chord_status_t chord_grouped_contiguous(const uint16_t* x, int64_t M, int K, const int32_t* m_indices,
                                         const void* w, int E, int N, uint16_t* out, void* workspace,
                                         size_t workspace_bytes, int flags, chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   if (M < 0) return fail(CHORD_ERR_INVALID_ARG, "M=%lld", (long long)M);
   const int64_t expected = E > 0 ? (M + E - 1) / E : 0;
   return grouped_gemm(x, M, K, m_indices, nullptr, 0, expected, w, E, N, out, workspace, workspace_bytes, flags,
@@ -446,7 +451,7 @@ chord_status_t chord_grouped_contiguous(const uint16_t* x, int64_t M, int K, con
 chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t max_m, int K, const int32_t* masked_m,
                                     int64_t expected_m, const void* w, int N, uint16_t* out, void* workspace,
                                     size_t workspace_bytes, int flags, chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   if (max_m < 1 || expected_m < 1)
     return fail(CHORD_ERR_INVALID_ARG, "max_m=%lld expected_m=%lld", (long long)max_m, (long long)expected_m);
   if (E < 1 || E > 1024) return fail(CHORD_ERR_UNSUPPORTED, "E=%d outside [1, 1024]", E);
@@ -456,7 +461,7 @@ chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t max_m, int
 }
 
 chord_status_t chord_set_timing_events(void* const* events, int n) {
-  g_detail[0] = 0;
+  clear_detail();
   if (n == 0) {
     g_timing_on = false;
     return CHORD_OK;
@@ -474,12 +479,11 @@ uint64_t chord_launch_count(void) { return g_launches.load(std::memory_order_rel
 
 chord_status_t chord_selftest_wait_timeout(uint32_t* status, uint64_t* elapsed_ns, uint32_t limit_us,
                                            chord_stream_t stream) {
-  g_detail[0] = 0;
+  clear_detail();
   if (!status || !elapsed_ns) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
   if (limit_us < 1 || limit_us > 1000000u)
     return fail(CHORD_ERR_INVALID_ARG, "limit_us must be in [1, 1000000], got %u", limit_us);
-  DeviceInfo dev;
-  chord_status_t st = current_device(&dev);
+  chord_status_t st = current_device(nullptr);
   if (st != CHORD_OK) return st;
   const cudaError_t err = launch_wait_timeout(status, elapsed_ns, uint64_t(limit_us) * 1000ull,
                                               reinterpret_cast<cudaStream_t>(stream));
@@ -487,7 +491,7 @@ chord_status_t chord_selftest_wait_timeout(uint32_t* status, uint64_t* elapsed_n
 }
 
 chord_status_t chord_moe_check_status(void* workspace, chord_stream_t stream_, uint32_t* device_status) {
-  g_detail[0] = 0;
+  clear_detail();
   if (!workspace) return fail(CHORD_ERR_INVALID_ARG, "null workspace");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   uint32_t v = 0;

@@ -111,6 +111,38 @@ __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int top
 }
 
 // ------------------------------------------------------------------------------------
+// Routing tag (num_tokens_padded[1]): the block_m the routing tensors were built for.
+
+__host__ __device__ constexpr int32_t routing_tag(int block_m) { return CHORD_ROUTING_TAG(block_m); }
+
+// The sorted positions a forward kernel may process: num_tokens_padded[0] clamped to
+// [0, cap], or 0 when num_tokens_padded[1] is not the tag of `block_m` (then
+// CHORD_DEV_BLOCK_M_MISMATCH is raised and no other routing tensor may be read: with a
+// smaller block_m than the routing sort used, expert_ids would be indexed past its end).
+__device__ __forceinline__ int routed_positions(const int32_t* ntp, int block_m, int64_t cap, uint32_t* status) {
+  if (ntp[1] != routing_tag(block_m)) {
+    atomicOr(status, CHORD_DEV_BLOCK_M_MISMATCH);
+    return 0;
+  }
+  int n = ntp[0];
+  if (n < 0) n = 0;
+  if (n > cap) n = int(cap);
+  return n;
+}
+
+// ------------------------------------------------------------------------------------
+// Host-side argument checks shared by the entry points (api.cu). fail() records the
+// detail text that chord_last_error_detail() returns and passes the status through.
+
+chord_status_t fail(chord_status_t st, const char* fmt, ...);
+chord_status_t cuda_fail(cudaError_t err, const char* what);
+void clear_detail();
+// T, topk, E and block_m of a routing sort: ranges and a capacity below 2^31.
+chord_status_t check_align_args(int64_t T, int topk, int E, int block_m);
+// The current device, which must be sm_100; *num_sms receives its SM count.
+chord_status_t current_device(int* num_sms);
+
+// ------------------------------------------------------------------------------------
 // PTX helpers (sm_100a)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -26,9 +26,12 @@ template <bool BLOCKED>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const int32_t* __restrict__ topk_ids, const float* __restrict__ topk_weights,
     const float* __restrict__ y, const int32_t* __restrict__ slot_pos, uint16_t* __restrict__ out, int64_t T,
-    int H, int topk, int E, int64_t cap) {
+    int H, int topk, int E, int64_t cap, const int32_t* __restrict__ ntp, int block_m) {
   grid_dep_wait();  // launched early: y comes from the down kernel
   const int lane = threadIdx.x & 31;
+  // routing built for another block_m: the GEMMs computed nothing, so every row is zero
+  // (the GEMM kernels raise CHORD_DEV_BLOCK_M_MISMATCH)
+  const bool routed = ntp[1] == routing_tag(block_m);
   const int nchunk = (H + kCombineCols - 1) / kCombineCols;
   for (int64_t item = blockIdx.x; item < T * nchunk; item += gridDim.x) {
     const int64_t t = item / nchunk;
@@ -43,7 +46,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
       if (j < topk) {
         const int64_t f = t * topk + j;
         const int e = __ldg(topk_ids + f);
-        if (unsigned(e) < unsigned(E)) {
+        if (routed && unsigned(e) < unsigned(E)) {
           w[h] = __ldg(topk_weights + f);
           if (BLOCKED) {
             const int pos = __ldg(slot_pos + f);
@@ -123,7 +126,10 @@ __global__ void validate_kernel(const int32_t* __restrict__ topk_ids,
                                 const int32_t* __restrict__ expert_ids,
                                 const int32_t* __restrict__ ntp_p, int block_m, int64_t cap,
                                 int64_t n_slots, int E, uint32_t* status) {
-  const int ntp = *ntp_p;
+  // another block_m's routing is reported by the GEMM kernels (CHORD_DEV_BLOCK_M_MISMATCH);
+  // its expert_ids may be shorter than this block_m's, so it is not read here
+  if (ntp_p[1] != routing_tag(block_m)) return;
+  const int ntp = ntp_p[0];
   if (ntp < 0 || ntp > cap || ntp % block_m != 0) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, CHORD_DEV_ROUTING_INVALID);
     return;
@@ -150,11 +156,11 @@ cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (a.y_blocked)
     err = launch_pdl(a.pdl, combine_kernel<true>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
                      a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
-                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap);
+                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap, a.ntp, a.block_m);
   else
     err = launch_pdl(a.pdl, combine_kernel<false>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
                      a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
-                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap);
+                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap, a.ntp, a.block_m);
   count_launches(1);
   return err != cudaSuccess ? err : cudaGetLastError();
 }

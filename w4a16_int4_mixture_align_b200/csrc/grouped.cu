@@ -133,7 +133,10 @@ __global__ void __launch_bounds__(kRouteThreads) grouped_route_masked_kernel(
               r + 2 < rows ? f + 2 : -1, r + 3 < rows ? f + 3 : -1);
     }
   }
-  if (tid == 0) *ntp = total * bm;
+  if (tid == 0) {
+    ntp[0] = total * bm;
+    ntp[1] = routing_tag(bm);
+  }
   if (__syncthreads_or(bad) && tid == 0) atomicOr(status, CHORD_DEV_ROUTING_INVALID);
 }
 
@@ -281,7 +284,10 @@ __global__ void __launch_bounds__(kRouteThreads) grouped_route_contiguous_kernel
     done += total;
     __syncthreads();  // the shared arrays are rewritten by the next batch
   }
-  if (tid == 0) *ntp = done * bm;
+  if (tid == 0) {
+    ntp[0] = done * bm;
+    ntp[1] = routing_tag(bm);
+  }
   if (__syncthreads_or(bad) && tid == 0) atomicOr(status, CHORD_DEV_ROUTING_INVALID);
 }
 

@@ -33,10 +33,9 @@ __device__ __forceinline__ void stg_stream(void* p, const uint4& v, uint64_t pol
 
 __global__ void __launch_bounds__(32 * kPermuteWarps) permute_rows_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ ntp_p,
-    int64_t cap, int64_t n_slots, int topk, int H, uint16_t* __restrict__ xs, int32_t* __restrict__ slot_pos) {
-  int64_t ntp = *ntp_p;
-  if (ntp < 0) ntp = 0;
-  if (ntp > cap) ntp = cap;
+    int block_m, int64_t cap, int64_t n_slots, int topk, int H, uint16_t* __restrict__ xs,
+    int32_t* __restrict__ slot_pos, uint32_t* __restrict__ status) {
+  const int64_t ntp = routed_positions(ntp_p, block_m, cap, status);
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = int64_t(blockIdx.x) * kPermuteWarps + (threadIdx.x >> 5);
   const int64_t nwarps = int64_t(gridDim.x) * kPermuteWarps;
@@ -69,9 +68,9 @@ cudaError_t launch_permute_rows(const ForwardArgs& a, cudaStream_t stream) {
   int64_t ctas = (a.cap + kPermuteWarps - 1) / kPermuteWarps;
   if (ctas > int64_t(a.num_sms) * 8) ctas = int64_t(a.num_sms) * 8;
   if (ctas < 1) ctas = 1;
-  permute_rows_kernel<<<unsigned(ctas), 32 * kPermuteWarps, 0, stream>>>(a.x, a.sorted_ids, a.ntp, a.cap,
+  permute_rows_kernel<<<unsigned(ctas), 32 * kPermuteWarps, 0, stream>>>(a.x, a.sorted_ids, a.ntp, a.block_m, a.cap,
                                                                          a.T * a.topk, a.topk, a.H, a.xs,
-                                                                         a.slot_pos);
+                                                                         a.slot_pos, a.status);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -207,9 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemm_kernel(StreamParams p
     // same wait) and the weights, so it starts streaming at once; its consumers wait for
     // the intermediate a.
     if (EPI != kDown) grid_dep_wait();
-    int ntp = *p.ntp;
-    if (ntp < 0) ntp = 0;
-    if (ntp > p.cap) ntp = int(p.cap);
+    const int ntp = routed_positions(p.ntp, p.block_m, p.cap, p.status);
     const int64_t nblocks = ntp / p.block_m;
     const int64_t items = nblocks * cpb * NGRP;
     const uint64_t pol_w = policy_evict_first();

@@ -266,9 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0) {
     // ----------------------------------------------------------------- activation producer
-    int ntp = *p.ntp;
-    if (ntp < 0) ntp = 0;
-    if (ntp > p.cap) ntp = int(p.cap);
+    const int ntp = routed_positions(p.ntp, p.block_m, p.cap, p.status);
     const int64_t nblocks = ntp / p.block_m;
     const int64_t items = nblocks * NT2;
     const uint64_t pol_a = policy_evict_last();
