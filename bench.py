@@ -2,26 +2,31 @@
 """Benchmark of the B200 W4A16 mixture-of-experts layer.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl chord|reference]
-                    [--workload ep8_decode|ep8_prefill|tp8_decode|tp8_prefill|skew|tiny
+                    [--workload all|ep8_decode|ep8_prefill|tp8_decode|tp8_prefill|skew|tiny
                                 |grouped_contiguous_ep8_gate_up|grouped_contiguous_ep8_down
                                 |grouped_masked_ep8_gate_up|grouped_masked_ep8_down]
 
 One step = one layer call through the C ABI: routing sort (chord_moe_align) then
-chord_moe_forward (gate_up GEMM + SiLU*up, down GEMM + top-k weight, combine), on a
-synthetic Kimi-K2-shaped batch already resident in HBM. The default workload is the
-EP8 decode shard: 128 tokens, hidden 7168, moe_intermediate 2048, experts 0..47 of
-384 local, top-8 from uniform router logits. Weights (1.19 GB) exceed the 126 MB L2,
-so no flush is needed between steps.
+chord_moe_forward (gate_up GEMM + SiLU*up, down GEMM, top-k weighted combine), on a
+synthetic Kimi-K2-shaped batch already resident in HBM. Weights (1.09-1.19 GB) exceed the
+126 MB L2, so no flush is needed between steps.
 
-Prints one JSON line (rank 0). `value` is microseconds per layer call for the whole job:
-the max over ranks of the timed region divided by (steps x ranks), since each rank runs
-an independent replica (the layer does not shard across GPUs here).
+By default (--workload all) every layer workload of the metric runs in turn -- EP8 decode,
+EP8 prefill, TP8 decode, TP8 prefill and the skewed-routing stress case -- each for K
+timed steps, and one JSON line is printed (rank 0): `value` is the EP8 decode shard
+(128 tokens, hidden 7168, moe_intermediate 2048, experts 0..47 of 384 local, top-8 from
+uniform router logits) in microseconds per layer call for the whole job, i.e. the max over
+ranks of the timed region divided by (steps x ranks), since each rank runs an independent
+replica (the layer does not shard across GPUs here); `per_workload` holds the same record
+for every workload: µs/call, per-kernel times, the roofline of the dominant kernel (HBM
+for the weight-streaming decode schedule, BF16 tensor for the tensor-core prefill one),
+the end-to-end number and the clocks seen.
 
 The grouped_* workloads time the grouped operators instead (one step = one
 chord_grouped_contiguous / chord_grouped_masked call: routing pass + GEMM) on an EP8 shard
 (48 experts) at the rows per expert the blog's grouped table uses.
 
---impl reference times the CPU oracle (test infrastructure) on the same workload on
+--impl reference times the CPU oracle (test infrastructure) on the headline workload on
 the host cores: rank 0 only, other ranks exit without work.
 """
 from __future__ import annotations
@@ -226,76 +231,104 @@ def pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world):
     return start.elapsed_time(stop)
 
 
-def run_chord(args, rank, world, local_rank):
+HEADLINE = "ep8_decode"
+LAYER_WORKLOADS = ["ep8_decode", "ep8_prefill", "tp8_decode", "tp8_prefill", "skew"]
+
+
+def tensor_peak(clocks, tf_burst, tf_sust, pk_kind):
+    """The BF16 denominator for a tensor-bound kernel, chosen from the run's own clock
+    record: the burst cuBLAS figure while the SM clock stays near its maximum, the
+    sustained (power-capped) figure only when the clock record shows it pulled down."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm and mx and sm < 0.9 * mx and "sw_power_cap" in clocks.get("reasons", []):
+        return tf_sust, f"{pk_kind} bf16_tflops_sustained (SM clock {sm:.0f} of {mx:.0f} MHz under sw_power_cap)"
+    return tf_burst, f"{pk_kind} bf16_tflops burst (SM clock {sm} of {mx} MHz)"
+
+
+class WeightCache:
+    """Repacked layers keyed by their weight shape: the EP8 workloads share one set of
+    weights (48 experts, intermediate 2048) and the TP8 ones another (384 experts, 256)."""
+
+    def __init__(self, dev):
+        self.dev, self.key, self.layer_args = dev, None, None
+
+    def get(self, cfg):
+        key = (cfg.E, cfg.H, cfg.I, cfg.seed)
+        if key != self.key:
+            self.layer_args = None
+            w = inputs.make_weights(cfg)
+            self.key, self.layer_args = key, (w[0], w[1].view(np.int16), w[2], w[3].view(np.int16))
+        return self.layer_args
+
+
+def run_workload(name, args, rank, world, local_rank, weights, sampler):
+    """One layer workload: `value` graph (K plain steps), an instrumented graph (K steps,
+    per-kernel events on every step) and the end-to-end leg; returns rank 0's record."""
     import torch
     from w4a16_int4_mixture_align_b200 import chord
 
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = inputs.CONFIGS[args.workload]
-    weights = inputs.make_weights(cfg)
+    cfg = inputs.CONFIGS[name]
     rcfg = inputs.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})  # each replica its own batch
     ids_np, tw_np = inputs.make_routing(rcfg)
     x_np = inputs.make_hidden(rcfg)
     work = algorithmic_work(cfg, ids_np)
-
-    layer = chord.ChordMoE(weights[0], weights[1].view(np.int16), weights[2], weights[3].view(np.int16),
-                           topk=cfg.topk, E_global=cfg.E_global, max_tokens=cfg.T, device=dev)
-    del weights
+    qw13, s13, qw2, s2 = weights.get(cfg)
+    layer = chord.ChordMoE(qw13, s13, qw2, s2, topk=cfg.topk, E_global=cfg.E_global, max_tokens=cfg.T, device=dev)
     x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
     ids = torch.from_numpy(ids_np).to(dev)
     tw = torch.from_numpy(tw_np).to(dev)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
-    # all GPU work of the timed leg runs on one side stream (graph capture needs one)
+    # all GPU work of the timed legs runs on one side stream (graph capture needs one)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
+    K = args.steps if args.steps is not None else DEFAULT_STEPS.get(name, 200)
+    W = args.warmup
 
     def step():
         layer.forward(x, ids, tw, out=out)
 
-    K, W = args.steps, args.warmup
     for _ in range(W):
         step()
     torch.cuda.synchronize()
     assert layer.check_status() == 0
 
-    # per-kernel events: [start, align done, gate_up done, down done, combine done] per step
+    # The K timed steps are captured once into a CUDA graph (the library enqueues
+    # everything on the caller's stream and never reads back, so a step is capturable),
+    # then replayed: the timed region runs exactly the K steps' kernels, without the host
+    # launch gaps of an eager loop, and with the early (programmatic) launches of the
+    # production path.
+    launches0 = chord.chord_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(K):
+            layer.align(ids)
+            chord.chord_moe_forward(x, ids, tw, layer.sorted_ids, layer.expert_ids, layer.ntp, layer.block_m,
+                                    layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace)
+    launches = chord.chord_launch_count() - launches0  # kernels per replay (captured once)
+    # The same K steps with the library's per-kernel timing events on every step: [start,
+    # align done, gate_up done, down done, combine done]. An event between two kernels
+    # orders them fully (no early launch), so these per-kernel times are each kernel's own
+    # duration, and their sum is a little above the production step time.
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(K)]
     for row in ev:
         for e in row:
             e.record(stream)
     torch.cuda.synchronize()
-
-    # The K timed steps are captured once into a CUDA graph (the library enqueues
-    # everything on the caller's stream and never reads back, so a step is capturable),
-    # then replayed: the timed region runs exactly the K steps' kernels, without the host
-    # launch gaps of an eager loop. Every EV_EVERY-th step also records the library's
-    # per-kernel timing events; an event node between two kernels turns off the early
-    # (programmatic) launch of the second, so only those steps pay for it, and `value`
-    # over all K steps stays slightly conservative.
-    timed_steps = [k for k in range(K) if k % EV_EVERY == 0]
-    launches0 = chord.chord_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
         for k in range(K):
-            timed = k % EV_EVERY == 0
-            if timed:
-                ev[k][0].record(stream)
+            ev[k][0].record(stream)
             layer.align(ids)
-            if timed:
-                chord.chord_set_timing_events(ev[k][1:5])
+            chord.chord_set_timing_events(ev[k][1:5])
             chord.chord_moe_forward(x, ids, tw, layer.sorted_ids, layer.expert_ids, layer.ntp, layer.block_m,
                                     layer.w13, layer.w2, layer.I, layer.E, out, layer.workspace)
-            if timed:
-                chord.chord_set_timing_events(None)
-    launches = chord.chord_launch_count() - launches0  # kernels per replay (captured once)
-    graph.replay()  # one untimed replay
+            chord.chord_set_timing_events(None)
+    graph.replay()  # one untimed replay of each
+    graph_ev.replay()
     torch.cuda.synchronize()
 
-    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
-    sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.25)  # a few clock samples before the timed region
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -307,11 +340,12 @@ def run_chord(args, rank, world, local_rank):
     t_wall1 = time.time()
     barrier(world)
     elapsed_ms = start.elapsed_time(stop)
+    graph_ev.replay()
+    torch.cuda.synchronize()
     assert layer.check_status() == 0
-    del graph
-
-    seg = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in timed_steps])
-    seg_ms = seg.mean(axis=0)  # align, gate_up, down, combine
+    del graph, graph_ev
+    seg = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in range(K)])
+    seg_ms = seg.mean(axis=0)  # align(+prep), gate_up, down, combine
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
@@ -335,69 +369,114 @@ def run_chord(args, rank, world, local_rank):
         out_h[s].copy_(outd[s].view(torch.int16), non_blocking=True)
 
     e2e_ms = pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world)
-    sampler.stop()
-
-    # ---- the fused router + routing sort at this workload's shape (outside the timed
-    # regions above; graph-replayed, so host marshalling does not hide device time)
-    router_us = time_router(chord, cfg, rcfg, dev)
     h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
     d2h = out_h[0].numel() * 2
+    router_us = time_router(chord, cfg, rcfg, dev) if name == HEADLINE else None
+    torch.cuda.set_stream(torch.cuda.default_stream(dev))
+    block_m = layer.block_m
+    del layer, xd, idsd, twd, outd
+    torch.cuda.empty_cache()
 
     # ---- max over ranks (outside the timed regions)
     stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
-    elapsed_ms, e2e_ms = stats[0], stats[1]
-    seg_ms = np.array(stats[2:])
+    elapsed_ms, e2e_ms, seg_ms = stats[0], stats[1], np.array(stats[2:])
     if rank != 0:
         return None
 
     hbm, tf_burst, tf_sust, pk_kind = peaks()
+    clocks = sampler.summary(t_wall0, t_wall1)
     us_call = job_us_per_call(elapsed_ms, K, world)
     gu_us, dn_us = seg_ms[1] * 1000.0, seg_ms[2] * 1000.0
-    decode = layer.block_m <= 32
+    decode = block_m <= 32
+    tf_peak, tf_src = tensor_peak(clocks, tf_burst, tf_sust, pk_kind)
     if decode:
         achieved = work["gate_up_bytes"] / (gu_us * 1e-6) / 1e9
+        achieved_dn = work["down_bytes"] / (dn_us * 1e-6) / 1e9
         roofline = {"bound": "hbm", "kernel": "stream_gemm gate_up", "achieved": round(achieved, 1),
                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                    "peak_source": f"{pk_kind} hbm_gbs",
-                    "traffic": recorded_traffic("stream_gemm_gate_up", args.workload),
-                    "algorithmic_bytes_per_launch": work["gate_up_bytes"]}
+                    "peak_source": f"{pk_kind} hbm_gbs (burst copy; kernel timed alone by its events)",
+                    "traffic": recorded_traffic("stream_gemm_gate_up", name),
+                    "algorithmic_bytes_per_launch": work["gate_up_bytes"],
+                    "down": {"achieved": round(achieved_dn, 1), "frac": round(achieved_dn / hbm, 4),
+                             "algorithmic_bytes_per_launch": work["down_bytes"]}}
     else:
-        # the GEMM is timed inside K back-to-back steps (hundreds of ms of tensor work under
-        # the power cap), so its denominator is the sustained cuBLAS figure; the burst
-        # fraction is reported beside it
         achieved = work["gate_up_flops"] / (gu_us * 1e-6) / 1e12
-        roofline = {"bound": "tensor", "kernel": "gate_up GEMM", "achieved": round(achieved, 1),
-                    "peak": tf_sust, "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
-                    "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long run of steps)",
-                    "peak_burst": tf_burst, "frac_of_burst": round(achieved / tf_burst, 4),
-                    "traffic": recorded_traffic("tc_gemm_gate_up", args.workload),
-                    "algorithmic_flops_per_launch": work["gate_up_flops"]}
+        achieved_dn = work["down_flops"] / (dn_us * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": "tc_gemm gate_up", "achieved": round(achieved, 1),
+                    "peak": tf_peak, "unit": "TFLOP/s", "frac": round(achieved / tf_peak, 4),
+                    "peak_source": tf_src,
+                    "frac_of_burst": round(achieved / tf_burst, 4), "frac_of_sustained": round(achieved / tf_sust, 4),
+                    "traffic": recorded_traffic("tc_gemm_gate_up", name),
+                    "algorithmic_flops_per_launch": work["gate_up_flops"],
+                    "down": {"achieved": round(achieved_dn, 1), "frac": round(achieved_dn / tf_peak, 4),
+                             "algorithmic_flops_per_launch": work["down_flops"]}}
     layer_us = elapsed_ms * 1000.0 / K
-    line = {
-        "metric": METRIC, "value": round(us_call, 3), "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": round(elapsed_ms / K, 5),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": describe(cfg), "block_m": layer.block_m,
-                   "schedule": "weight-streaming" if decode else "tensor-core",
-                   "routed_pairs": work["R"], "active_experts": work["active_experts"],
-                   "l2": "no flush: weights %.2f GB > 126 MB L2" % (work["layer_bytes"] / 1e9),
-                   "parallelism": f"replicas x{world}"},
+    rec = {
+        "workload": describe(cfg), "us_per_call": round(us_call, 3), "steps": K, "warmup": W,
+        "block_m": block_m, "schedule": "weight-streaming" if decode else "tensor-core",
+        "routed_pairs": work["R"], "active_experts": work["active_experts"],
+        "l2": "no flush: weights %.2f GB > 126 MB L2" % (work["layer_bytes"] / 1e9),
         "kernels_us": {"align+prep": round(seg_ms[0] * 1000, 2), "gate_up": round(gu_us, 2),
                        "down": round(dn_us, 2), "combine": round(seg_ms[3] * 1000, 2),
-                       "gate_up+down": round(gu_us + dn_us, 2)},
+                       "gate_up+down": round(gu_us + dn_us, 2),
+                       "how": "each kernel alone: CUDA events around it on every step of an "
+                              "instrumented replay of the same K steps (no early launch)"},
         "layer": {"GB/s": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9, 1),
                   "hbm_frac": round(work["layer_bytes"] / (layer_us * 1e-6) / 1e9 / hbm, 4),
-                  "TFLOP/s": round((work["gate_up_flops"] + work["down_flops"]) / (layer_us * 1e-6) / 1e12, 2)},
+                  "TFLOP/s": round((work["gate_up_flops"] + work["down_flops"]) / (layer_us * 1e-6) / 1e12, 2),
+                  "tensor_frac": round((work["gate_up_flops"] + work["down_flops"]) / (layer_us * 1e-6) / 1e12
+                                       / tf_peak, 4)},
         "roofline": roofline,
         "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
-        "clocks": sampler.summary(t_wall0, t_wall1),
-        "router_topk_align": {"us_per_call": round(router_us, 2),
-                              "what": "chord_router_topk_align on fp32 logits [T, E_global], top-%d, "
-                                      "then the routing sort (not part of value)" % cfg.topk},
+        "clocks": clocks,
     }
+    if router_us is not None:
+        rec["router_topk_align"] = {
+            "us_per_call": round(router_us, 2),
+            "what": "chord_router_topk_align on fp32 logits [T, E_global], top-%d, then the routing sort "
+                    "(not part of value)" % cfg.topk}
+    return rec
+
+
+def run_chord(args, rank, world, local_rank):
+    """The layer workloads: the headline (EP8 decode) as `value`, every workload of the
+    metric in `per_workload` (or one workload when --workload names it)."""
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    names = LAYER_WORKLOADS if args.workload == "all" else [args.workload]
+    head = HEADLINE if args.workload == "all" else args.workload
+    weights = WeightCache(dev)
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
+    sampler.start()
+    recs = {}
+    try:
+        for name in names:
+            recs[name] = run_workload(name, args, rank, world, local_rank, weights, sampler)
+    finally:
+        sampler.stop()
+    if rank != 0:
+        return None
+    h = recs[head]
+    cfg = inputs.CONFIGS[head]
+    line = {
+        "metric": METRIC, "value": h["us_per_call"], "unit": UNIT, "n_gpus": world,
+        "steps": h["steps"], "warmup": h["warmup"], "ms_per_step": round(h["us_per_call"] * world / 1000.0, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "block_m": h["block_m"], "schedule": h["schedule"],
+                   "routed_pairs": h["routed_pairs"], "active_experts": h["active_experts"],
+                   "l2": h["l2"], "parallelism": f"replicas x{world}"},
+        "kernels_us": h["kernels_us"], "layer": h["layer"], "roofline": h["roofline"], "e2e": h["e2e"],
+        "gpu_launches": h["gpu_launches"], "clocks": h["clocks"],
+    }
+    if "router_topk_align" in h:
+        line["router_topk_align"] = h["router_topk_align"]
+    if len(recs) > 1:
+        line["per_workload"] = recs
     return line
 
 
@@ -680,7 +759,7 @@ def run_reference(args, rank, world):
     oracle.build()
     if args.workload in inputs.GROUPED_CONFIGS:
         return run_reference_grouped(args, world)
-    cfg = inputs.CONFIGS[args.workload]
+    cfg = inputs.CONFIGS[HEADLINE if args.workload == "all" else args.workload]
     d = inputs.make_inputs(cfg)
     threads = os.cpu_count() or 1
     for _ in range(args.warmup):
@@ -729,16 +808,17 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["chord", "reference"], default="chord")
-    ap.add_argument("--workload", choices=list(inputs.CONFIGS) + sorted(inputs.GROUPED_CONFIGS),
-                    default="ep8_decode")
+    ap.add_argument("--workload", choices=["all"] + list(inputs.CONFIGS) + sorted(inputs.GROUPED_CONFIGS),
+                    default="all",
+                    help="all (default): the EP8 decode headline plus every layer workload of the metric")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=["auto", "stream", "tensor"], default="auto",
                     help="grouped workloads: force the GEMM schedule")
     ap.add_argument("--expected-m", type=int, default=None,
                     help="grouped masked workloads: the expected_m hint (default: the rows per expert)")
     args = ap.parse_args()
-    if args.steps is None:
-        args.steps = 3 if args.impl == "reference" else DEFAULT_STEPS.get(args.workload, 200)
+    if args.steps is None and (args.impl == "reference" or args.workload in inputs.GROUPED_CONFIGS):
+        args.steps = 3 if args.impl == "reference" else 200
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -763,7 +843,8 @@ def main():
     if line is not None:
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = (grouped_cpu_baseline(inputs.GROUPED_CONFIGS[args.workload]) if grouped
-                                    else cpu_baseline(inputs.CONFIGS[args.workload]))
+                                    else cpu_baseline(inputs.CONFIGS[HEADLINE if args.workload == "all"
+                                                                         else args.workload]))
         else:
             line["cpu_baseline"] = None
     if world > 1:

@@ -72,6 +72,10 @@ typedef enum {
  * other than this library must write it too. */
 #define CHORD_ROUTING_TAG(block_m) ((int32_t)(0x52540000u | (uint32_t)(block_m)))
 
+/* Bytes at the start of a forward or grouped workspace that the caller zeroes once after
+ * allocating it (status word and stream-K flags); the library keeps them consistent. */
+#define CHORD_WORKSPACE_HEADER_BYTES 65536
+
 /* Weight roles for chord_repack_weights. */
 #define CHORD_ROLE_GATE_UP 1 /* W13 [E, 2I, H]: rows [0,I) gate, rows [I,2I) up */
 #define CHORD_ROLE_DOWN    2 /* W2  [E, H, I] */
@@ -221,9 +225,11 @@ CHORD_API int chord_select_block_m(int64_t T, int topk, int E_local, int E_globa
  *              captured graph needs no readback).
  * w13, w2      device blobs from chord_repack_weights (roles GATE_UP [E,2I,H], DOWN [E,H,I])
  * out          device bf16 [T, H]; every row is written (0 for tokens with no local slot)
- * workspace    device, >= chord_moe_workspace_bytes(), 256-byte aligned. Its first 256
- *              bytes hold the device status word: zero them once after allocating; the
- *              rest is scratch that needs no initialisation.
+ * workspace    device, >= chord_moe_workspace_bytes(), 256-byte aligned. Its first
+ *              CHORD_WORKSPACE_HEADER_BYTES hold the device status word (offset 0) and the
+ *              flags with which the weight-streaming GEMM's stream-K workers hand partial
+ *              sums to one another (each flag is reset by its reader): zero them once after
+ *              allocating. The rest is scratch that needs no initialisation.
  *
  * Requires H % 128 == 0, I % 128 == 0, 1 <= block_m <= 256 (same as used for align).
  * Concurrent forwards must not share a workspace.
@@ -272,8 +278,9 @@ CHORD_API chord_status_t chord_moe_check_status(void* workspace, chord_stream_t 
  *   process) or sets CHORD_DEV_BLOB_MISMATCH (foreign blob: the kernel reads its
  *   header). N % 128 == 0, K % 128 == 0, 1 <= E <= 1024.
  *   workspace: device, >= chord_grouped_workspace_bytes(rows, E) bytes, rows = M or
- *   E * max_m, 256-byte aligned; its first 256 bytes hold the status word as for
- *   chord_moe_forward (zero once; read with chord_moe_check_status).
+ *   E * max_m, 256-byte aligned; its first CHORD_WORKSPACE_HEADER_BYTES hold the status
+ *   word and the stream-K flags as for chord_moe_forward (zero once; read the status with
+ *   chord_moe_check_status).
  *   flags: CHORD_FLAG_FORCE_STREAM / CHORD_FLAG_FORCE_TENSOR pick the schedule; by
  *   default expected rows per expert (M / E, or expected_m) <= 16 streams the weights.
  *   Two kernels run on `stream`: a routing pass over m_indices / masked_m, then the GEMM;

@@ -19,9 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libchord.so")
-SOURCES = ["api.cu", "align.cu", "align_static.cu", "repack.cu", "stream_gemm.cu", "tc_gemm.cu", "permute.cu", "grouped.cu",
+SOURCES = ["api.cu", "align.cu", "align_static.cu", "repack.cu", "stream_gemm.cu", "stream_gemm_short.cu", "tc_gemm.cu", "permute.cu", "grouped.cu",
            "combine.cu", "diag.cu"]
-HEADERS = ["chord_internal.cuh", "tc_common.cuh"]
+HEADERS = ["chord_internal.cuh", "tc_common.cuh", "stream_common.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -322,6 +322,9 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   a.xs = reinterpret_cast<uint16_t*>(wsb + ws.xs_offset);
   a.slot_pos = reinterpret_cast<int32_t*>(wsb + ws.slot_pos_offset);
   a.status = reinterpret_cast<uint32_t*>(wsb);
+  a.stream_flags = reinterpret_cast<uint32_t*>(wsb + ws.flags_offset);
+  a.stream_partial = reinterpret_cast<float*>(wsb + ws.partial_offset);
+  a.stream_partial_bytes = ws.partial_bytes;
   a.T = T;
   a.H = H;
   a.I = I;
@@ -422,6 +425,8 @@ chord_status_t grouped_gemm(const uint16_t* x, int64_t rows, int K, const int32_
   g.bm = bm;
   g.cap = ws.max_positions;
   g.status = reinterpret_cast<uint32_t*>(wsb);
+  g.stream_flags = reinterpret_cast<uint32_t*>(wsb + ws.flags_offset);
+  g.stream_partial = reinterpret_cast<float*>(wsb + ws.partial_offset);
   g.num_sms = num_sms;
   cudaError_t err = launch_grouped_route(m_indices, rows, masked_m, E, max_m, bm,
                                          const_cast<int32_t*>(g.expert_ids), const_cast<int32_t*>(g.block_row0),

@@ -87,8 +87,27 @@ __host__ __device__ inline int code_slot(int g, int t) { return t ^ ((g >> 1) & 
 __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1); }
 
 // ------------------------------------------------------------------------------------
+// Stream-K scratch of the weight-streaming GEMM: each of its workers (two consumer groups
+// per CTA, at most kMaxStreamCtas CTAs) may leave one FP32 partial tile (8 warps x 32
+// lanes x TC/2 floats) behind, announced by one flag per warp. Flags are zero between
+// launches (each is reset by the worker that consumes it), so they live in the
+// workspace header, which the caller zeroes once.
+constexpr int kMaxStreamCtas = 256;
+constexpr int kMaxStreamWorkers = 2 * kMaxStreamCtas;
+constexpr uint64_t kStreamFlagBytes = uint64_t(kMaxStreamWorkers) * 8 * 4;
+__host__ __device__ inline int stream_token_chunk(int block_m) { return block_m <= 8 ? 8 : (block_m <= 16 ? 16 : 32); }
+__host__ __device__ inline uint64_t stream_partial_bytes(int tc) {
+  return uint64_t(kMaxStreamWorkers) * 8 * 32 * (tc / 2) * 4;
+}
+// Header of both workspaces (forward and grouped): the device status word at offset 0,
+// the stream-K flags from offset 256. Zeroed once by the caller after allocation.
+constexpr uint64_t kWorkspaceHeaderBytes = CHORD_WORKSPACE_HEADER_BYTES;
+static_assert(256 + 2 * kStreamFlagBytes <= kWorkspaceHeaderBytes, "workspace header");
+
 // Workspace of chord_moe_forward:
-//   [status 256 B][a: cap x I bf16][y: cap x H fp32][xs: cap x H bf16][slot_pos: T*topk i32]
+//   [header 64 KiB: status, stream-K flags of the gate_up and down GEMMs]
+//   [a: cap x I bf16][y: cap x H fp32][xs: cap x H bf16][slot_pos: T*topk i32]
+//   [stream-K partials of the gate_up and down GEMMs]
 // a is the SiLU*up intermediate by sorted position (row-major [cap, I]); y the expert outputs
 // before the top-k weight (by flat slot [T*topk, H] on the streaming schedule, by sorted
 // position in 128-column blocks [H/128][cap][128] on the tensor-core schedule, so that a
@@ -96,17 +115,20 @@ __host__ __device__ inline int nibble_slot(int u) { return (u >> 1) + 4 * (u & 1
 // and slot_pos the sorted position of every local flat slot (both tensor-core schedule
 // only).
 struct ForwardWorkspace {
-  uint64_t a_offset, y_offset, xs_offset, slot_pos_offset, total;
+  uint64_t flags_offset, a_offset, y_offset, xs_offset, slot_pos_offset, partial_offset, partial_bytes, total;
 };
 __host__ __device__ inline ForwardWorkspace forward_workspace(int64_t T, int topk, int E, int H,
                                                               int I, int block_m) {
   ForwardWorkspace w;
   int64_t cap = T * topk + int64_t(E) * (block_m - 1);
-  w.a_offset = 256;
+  w.flags_offset = 256;  // [2][kMaxStreamWorkers][8]: gate_up, down
+  w.a_offset = kWorkspaceHeaderBytes;
   w.y_offset = align256(w.a_offset + uint64_t(cap) * I * 2);
   w.xs_offset = align256(w.y_offset + uint64_t(cap) * H * 4);
   w.slot_pos_offset = align256(w.xs_offset + uint64_t(cap) * H * 2);
-  w.total = align256(w.slot_pos_offset + uint64_t(T) * topk * 4);
+  w.partial_offset = align256(w.slot_pos_offset + uint64_t(T) * topk * 4);
+  w.partial_bytes = stream_partial_bytes(stream_token_chunk(block_m));  // per GEMM
+  w.total = align256(w.partial_offset + 2 * w.partial_bytes);
   return w;
 }
 
@@ -395,6 +417,9 @@ struct ForwardArgs {
   bool y_blocked;     // y is by sorted position in 128-column blocks
   bool pdl;           // launch the streaming GEMMs and the combine early (programmatic)
   uint32_t* status;
+  uint32_t* stream_flags;   // [2][kMaxStreamWorkers][8] stream-K flags (gate_up, down)
+  float* stream_partial;    // [2] x stream_partial_bytes stream-K partials (gate_up, down)
+  uint64_t stream_partial_bytes;
   int64_t T;
   int H, I, E, topk, block_m;
   int64_t cap;     // sorted_ids capacity
@@ -404,7 +429,8 @@ struct ForwardArgs {
 // Grouped operators: workspace layout for `rows` rows of x (M, or E * max_m) and E
 // experts, for any unit size bm in {8, 16, 32, 64, 128, 256}.
 struct GroupedWorkspace {
-  int64_t max_units, max_positions, ntp_offset, expert_ids_offset, block_row0_offset, sorted_ids_offset, total;
+  int64_t max_units, max_positions, flags_offset, ntp_offset, expert_ids_offset, block_row0_offset, sorted_ids_offset,
+      partial_offset, total;
 };
 GroupedWorkspace grouped_workspace(int64_t rows, int E);
 // The routing pass: m_indices (contiguous, 16-byte aligned) or masked_m (masked) -> units
@@ -426,6 +452,8 @@ struct GroupedArgs {
   int bm;                   // positions per unit
   int64_t cap;              // sorted_ids capacity
   uint32_t* status;
+  uint32_t* stream_flags;   // [kMaxStreamWorkers][8] stream-K flags
+  float* stream_partial;    // stream-K partials (token chunk up to 32)
   int num_sms;
 };
 // The GEMM of the grouped operators: out[row] = x[row] . W[e]^T for every valid row.

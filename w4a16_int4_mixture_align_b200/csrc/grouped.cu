@@ -300,11 +300,13 @@ GroupedWorkspace grouped_workspace(int64_t rows, int E) {
   w.max_units = (rows + 7) / 8 + E;
   w.max_positions = ((rows + 127) / 128 + E) * 256;
   auto up = [](int64_t b) { return (b + 255) / 256 * 256; };
-  w.ntp_offset = 256;
+  w.flags_offset = 256;  // stream-K flags, inside the zero-once header
+  w.ntp_offset = int64_t(kWorkspaceHeaderBytes);
   w.expert_ids_offset = w.ntp_offset + 256;
   w.block_row0_offset = w.expert_ids_offset + up(w.max_units * 4);
   w.sorted_ids_offset = w.block_row0_offset + up(w.max_units * 4);
-  w.total = w.sorted_ids_offset + up(w.max_positions * 4);
+  w.partial_offset = w.sorted_ids_offset + up(w.max_positions * 4);
+  w.total = w.partial_offset + int64_t(stream_partial_bytes(32));
   return w;
 }
 
