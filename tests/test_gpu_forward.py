@@ -241,3 +241,27 @@ def test_block_m_mismatch_is_caught_on_the_device(chord, tiny, path, bm_align, b
     # the matching block_m on the same buffers still computes the layer
     got = run_layer(dst, tiny, flags)
     assert_layer_close(got, oracle_rows(tiny, None))
+
+
+# ------------------------------------------------------------------------------ full size, other schedules
+
+@pytest.mark.parametrize("name,block_m,flags", [
+    ("tp8_prefill", 64, 0),     # tensor cores, an expert's ~85 rows in two 64-row blocks
+    ("tp8_prefill", 96, 0),     # tensor cores, MMA N of a block not a power of two
+    ("ep8_prefill", 64, 0),     # tensor cores, ~171 rows per expert in three blocks
+    ("ep8_prefill", 96, 0),
+    ("tp8_prefill", 128, "stream"),  # weight streaming at a prefill shape: 32-token chunks
+    ("ep8_decode", 32, "tensor"),    # tensor cores at a decode shape
+])
+def test_full_size_other_block_m_and_forced_schedules(chord, big_inputs, name, block_m, flags):
+    # the selector's own choice is covered by test_full_size_sampled_rows; these are the
+    # block sizes and schedules a caller may pick at Kimi-K2 sizes
+    d = big_inputs(name)
+    cfg = d["cfg"]
+    f = {0: 0, "stream": chord.CHORD_FLAG_FORCE_STREAM, "tensor": chord.CHORD_FLAG_FORCE_TENSOR}[flags]
+    layer = make_layer(chord, d, block_m=block_m)
+    got = run_layer(layer, d, f)
+    rows = inputs.sample_rows(d["topk_ids"], cfg.E, 512, seed=1)
+    assert_layer_close(got[rows], oracle_rows(d, rows))
+    none = ~((d["topk_ids"] >= 0) & (d["topk_ids"] < cfg.E)).any(axis=1)
+    assert np.all(bf16_bits_to_f64(got[none]) == 0)
