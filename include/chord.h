@@ -86,6 +86,8 @@ typedef enum {
 #define CHORD_FLAG_VALIDATE_ROUTING 0x1 /* check routing tensors on the device first */
 #define CHORD_FLAG_FORCE_STREAM     0x2 /* force the weight-streaming (decode) schedule */
 #define CHORD_FLAG_FORCE_TENSOR     0x4 /* force the tensor-core (prefill) schedule */
+#define CHORD_FLAG_OUTPUT_FP32      0x8 /* `out` is float [T, H]: the FP32 sums before the final
+                                           BF16 rounding (a tensor-parallel rank's partial) */
 
 CHORD_API const char* chord_status_string(int status);
 CHORD_API const char* chord_last_error_detail(void);
@@ -294,6 +296,52 @@ CHORD_API chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t 
                                               const int32_t* masked_m, int64_t expected_m, const void* w, int N,
                                               uint16_t* out, void* workspace, size_t workspace_bytes, int flags,
                                               chord_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Exchange steps of sharded deployments. The Chord blog runs the layer as expert-parallel
+ * (EP8/EP16/EP32) and tensor-parallel (TP8 single-instance) shards ("TL;DR";
+ * "vLLM-Integration": the h200_tp8 profile) and leaves the communication out of its
+ * kernel timings ("Messungen"). These entry points are the device steps around the
+ * collectives; the collectives themselves (all-to-all, all-reduce) are the caller's.
+ *
+ * Expert parallel, W ranks, rank d owning global experts [d*E_rank, (d+1)*E_rank):
+ *  chord_ep_plan: for this rank's T tokens and their GLOBAL topk_ids [T, topk] (ids outside
+ *    [0, W*E_rank) are dropped), one send row per (token t, rank d) such that t has at
+ *    least one slot on d. send_rows[i] = t*W + d for the i-th send row, rows grouped by
+ *    d in increasing d and by t in increasing t inside each group; rank_offsets[d] = the
+ *    first row of rank d, rank_offsets[W] = the row count (the caller reads the W + 1
+ *    offsets back to size its all-to-all); row_of[t*W + d] = -1 for every pair (set here,
+ *    filled by chord_ep_pack). send_rows: device int32 [T*W]; rank_offsets: device int32
+ *    [W+1]; row_of: device int32 [T*W]; workspace: device, >= chord_ep_plan_workspace_bytes,
+ *    256-byte aligned, scratch. Limits: 1 <= W <= 64, W*E_rank <= 4096, T*W < 2^31.
+ *  chord_ep_pack: the send buffers of those rows: send_x[i] = hidden[t] (bf16 [rows, H]),
+ *    send_ids[i, j] = topk_ids[t, j] - d*E_rank when slot j is on rank d, else -1, and
+ *    send_w[i, j] = topk_weights[t, j] for those slots, else 0; row_of[t*W + d] = i. The
+ *    receiving rank runs chord_moe_align + chord_moe_forward on the rows it receives (with
+ *    send_ids as topk_ids over its E_rank experts) and returns one bf16 output row per row.
+ *    send_x: device bf16 [T*W, H] (capacity), send_ids int32 / send_w fp32 [T*W, topk];
+ *    hidden and send_x 16-byte aligned, H % 8 == 0.
+ *  chord_ep_combine: out[t] = bf16( sum over d = 0 .. W-1 with a row i = row_of[t*W + d]
+ *    of float(back[i]) ), the sum in FP32 in increasing d; 0 for a token with no slot on
+ *    any rank. back: device bf16 [rows, H], the returned rows in send-row order; out:
+ *    device bf16 [T, H]; both 16-byte aligned.
+ * Tensor parallel, each rank holding a slice of every expert's intermediate dimension:
+ *  chord_moe_forward with CHORD_FLAG_OUTPUT_FP32 writes the rank's FP32 partial output,
+ *  the caller all-reduces the partials (sum), and chord_round_bf16 rounds the total once:
+ *  out[i] = bf16_rne(in[i]) for i < n (device float in, device bf16 out).
+ * All are asynchronous on `stream`; argument errors return before anything is enqueued.
+ * ---------------------------------------------------------------------------------- */
+CHORD_API size_t chord_ep_plan_workspace_bytes(int64_t T, int W);
+CHORD_API chord_status_t chord_ep_plan(const int32_t* topk_ids, int64_t T, int topk, int E_rank, int W,
+                                       int32_t* send_rows, int32_t* rank_offsets, int32_t* row_of, void* workspace,
+                                       size_t workspace_bytes, chord_stream_t stream);
+CHORD_API chord_status_t chord_ep_pack(const uint16_t* hidden, const int32_t* topk_ids, const float* topk_weights,
+                                       int64_t T, int H, int topk, int E_rank, int W, const int32_t* send_rows,
+                                       const int32_t* rank_offsets, int32_t* row_of, uint16_t* send_x,
+                                       int32_t* send_ids, float* send_w, chord_stream_t stream);
+CHORD_API chord_status_t chord_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t T, int H, int W,
+                                          uint16_t* out, chord_stream_t stream);
+CHORD_API chord_status_t chord_round_bf16(const float* in, int64_t n, uint16_t* out, chord_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used by the benchmark).

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libchord.so")
-SOURCES = ["api.cu", "align.cu", "align_static.cu", "repack.cu", "stream_gemm.cu", "stream_gemm_short.cu", "tc_gemm.cu", "permute.cu", "grouped.cu",
+SOURCES = ["api.cu", "align.cu", "align_static.cu", "repack.cu", "stream_gemm.cu", "stream_gemm_short.cu", "tc_gemm.cu", "permute.cu", "grouped.cu", "shard.cu",
            "combine.cu", "diag.cu"]
 HEADERS = ["chord_internal.cuh", "tc_common.cuh", "stream_common.cuh"]
 

@@ -41,6 +41,7 @@ CHORD_ROLE_GROUPED_MASKED = 4
 CHORD_FLAG_VALIDATE_ROUTING = 0x1
 CHORD_FLAG_FORCE_STREAM = 0x2
 CHORD_FLAG_FORCE_TENSOR = 0x4
+CHORD_FLAG_OUTPUT_FP32 = 0x8
 
 # every symbol include/chord.h declares: (name, restype, argtypes)
 _P = ctypes.c_void_p
@@ -67,6 +68,11 @@ SIGNATURES = {
     "chord_grouped_workspace_bytes": (_SZ, [_I64, _I]),
     "chord_grouped_contiguous": (_I, [_P, _I64, _I, _P, _P, _I, _I, _P, _P, _SZ, _I, _P]),
     "chord_grouped_masked": (_I, [_P, _I, _I64, _I, _P, _I64, _P, _I, _P, _P, _SZ, _I, _P]),
+    "chord_ep_plan_workspace_bytes": (_SZ, [_I64, _I]),
+    "chord_ep_plan": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "chord_ep_pack": (_I, [_P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "chord_ep_combine": (_I, [_P, _P, _I64, _I, _I, _P, _P]),
+    "chord_round_bf16": (_I, [_P, _I64, _P, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
     "chord_selftest_wait_timeout": (_I, [_P, _P, ctypes.c_uint32, _P]),
@@ -233,6 +239,38 @@ def chord_grouped_masked(x, masked_m, expected_m, w, N, out, workspace, flags=0,
     _check(lib().chord_grouped_masked(_ptr(x), E, max_m, K, _ptr(masked_m), int(expected_m), _ptr(w), N,
                                       _ptr(out), _ptr(workspace), _nbytes(workspace), flags, _stream(stream)),
            "chord_grouped_masked")
+
+
+def chord_ep_plan_workspace_bytes(T, W) -> int:
+    return int(lib().chord_ep_plan_workspace_bytes(T, W))
+
+
+def chord_ep_plan(topk_ids, E_rank, W, send_rows, rank_offsets, row_of, workspace, stream=None):
+    """Expert-parallel send plan: one row per (token, rank owning >= 1 of its experts),
+    grouped by rank; rank_offsets [W+1]; row_of [T*W] reset to -1."""
+    T, topk = topk_ids.shape
+    _check(lib().chord_ep_plan(_ptr(topk_ids), T, topk, E_rank, W, _ptr(send_rows), _ptr(rank_offsets), _ptr(row_of),
+                               _ptr(workspace), _nbytes(workspace), _stream(stream)), "chord_ep_plan")
+
+
+def chord_ep_pack(hidden, topk_ids, topk_weights, E_rank, W, send_rows, rank_offsets, row_of, send_x, send_ids,
+                  send_w, stream=None):
+    T, H = hidden.shape
+    topk = topk_ids.shape[1]
+    _check(lib().chord_ep_pack(_ptr(hidden), _ptr(topk_ids), _ptr(topk_weights), T, H, topk, E_rank, W,
+                               _ptr(send_rows), _ptr(rank_offsets), _ptr(row_of), _ptr(send_x), _ptr(send_ids),
+                               _ptr(send_w), _stream(stream)), "chord_ep_pack")
+
+
+def chord_ep_combine(back, row_of, W, out, stream=None):
+    T, H = out.shape
+    _check(lib().chord_ep_combine(_ptr(back) if back.numel() else None, _ptr(row_of), T, H, W, _ptr(out),
+                                  _stream(stream)), "chord_ep_combine")
+
+
+def chord_round_bf16(x_f32, out_bf16, stream=None):
+    assert x_f32.dtype == torch.float32 and x_f32.numel() == out_bf16.numel()
+    _check(lib().chord_round_bf16(_ptr(x_f32), x_f32.numel(), _ptr(out_bf16), _stream(stream)), "chord_round_bf16")
 
 
 def chord_moe_check_status(workspace, stream=None) -> int:

@@ -343,6 +343,7 @@ chord_status_t chord_moe_forward(const uint16_t* hidden, const int32_t* topk_ids
   const bool tensor = (flags & CHORD_FLAG_FORCE_TENSOR) ||
                       (!(flags & CHORD_FLAG_FORCE_STREAM) && block_m > 32);
   a.y_blocked = tensor;
+  a.out_f32 = (flags & CHORD_FLAG_OUTPUT_FP32) != 0;
   // early (programmatic) launches on the weight-streaming schedule; not while timing events
   // are recorded between the kernels (an event between two kernels orders them fully)
   a.pdl = !tensor && !timing;
@@ -463,6 +464,121 @@ chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t max_m, int
   if (!masked_m) return fail(CHORD_ERR_INVALID_ARG, "null masked_m");
   return grouped_gemm(x, int64_t(E) * max_m, K, nullptr, masked_m, max_m, expected_m, w, E, N, out, workspace,
                       workspace_bytes, flags, CHORD_ROLE_GROUPED_MASKED, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------------------------
+// Exchange steps of sharded deployments
+
+namespace {
+
+chord_status_t check_ep_args(int64_t T, int topk, int E_rank, int W) {
+  if (T < 0 || topk < 1 || topk > 64) return fail(CHORD_ERR_INVALID_ARG, "T=%lld topk=%d", (long long)T, topk);
+  if (W < 1 || W > 64) return fail(CHORD_ERR_UNSUPPORTED, "W=%d ranks outside [1, 64]", W);
+  if (E_rank < 1 || int64_t(E_rank) * W > 4096)
+    return fail(CHORD_ERR_UNSUPPORTED, "E_rank=%d x W=%d experts outside [1, 4096]", E_rank, W);
+  if (T >= (int64_t(1) << 31) / W) return fail(CHORD_ERR_UNSUPPORTED, "T*W >= 2^31");
+  return CHORD_OK;
+}
+
+struct EpPlanWorkspace {
+  uint64_t ids_offset, expert_ids_offset, ntp_offset, align_offset, total;
+};
+EpPlanWorkspace ep_plan_workspace(int64_t T, int W) {
+  EpPlanWorkspace w;
+  const uint64_t n = uint64_t(T) * W;
+  w.ids_offset = 0;
+  w.expert_ids_offset = align256(n * 4);
+  w.ntp_offset = w.expert_ids_offset + align256(n * 4 > 0 ? n * 4 : 4);
+  w.align_offset = w.ntp_offset + 256;
+  w.total = w.align_offset + align256(align_workspace_bytes(int64_t(n), W));
+  return w;
+}
+
+}  // namespace
+
+size_t chord_ep_plan_workspace_bytes(int64_t T, int W) {
+  if (T < 0 || W < 1) return 0;
+  return size_t(ep_plan_workspace(T, W).total);
+}
+
+chord_status_t chord_ep_plan(const int32_t* topk_ids, int64_t T, int topk, int E_rank, int W, int32_t* send_rows,
+                             int32_t* rank_offsets, int32_t* row_of, void* workspace, size_t workspace_bytes,
+                             chord_stream_t stream) {
+  clear_detail();
+  chord_status_t st = check_ep_args(T, topk, E_rank, W);
+  if (st != CHORD_OK) return st;
+  if ((T > 0 && (!topk_ids || !send_rows || !row_of)) || !rank_offsets || !workspace)
+    return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if (!aligned256(workspace)) return fail(CHORD_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const EpPlanWorkspace ws = ep_plan_workspace(T, W);
+  if (workspace_bytes < ws.total)
+    return fail(CHORD_ERR_WORKSPACE_TOO_SMALL, "ep plan workspace needs %llu bytes, got %zu",
+                (unsigned long long)ws.total, workspace_bytes);
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  int32_t* ids_tw = reinterpret_cast<int32_t*>(wsb + ws.ids_offset);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  if (T > 0) err = launch_ep_route(topk_ids, T, topk, E_rank, W, ids_tw, row_of, num_sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "ep route launch");
+  // the routing sort over W "experts" (the ranks) with blocks of one row: rows grouped by
+  // destination, ascending token inside each, and the per-rank offsets
+  const int64_t n = T * W;
+  err = launch_align(ids_tw, n, W, 1, n, n, send_rows ? send_rows : ids_tw,
+                     reinterpret_cast<int32_t*>(wsb + ws.expert_ids_offset), reinterpret_cast<int32_t*>(wsb + ws.ntp_offset),
+                     rank_offsets, wsb + ws.align_offset, s);
+  if (err != cudaSuccess) return cuda_fail(err, "ep plan sort launch");
+  return CHORD_OK;
+}
+
+chord_status_t chord_ep_pack(const uint16_t* hidden, const int32_t* topk_ids, const float* topk_weights, int64_t T,
+                             int H, int topk, int E_rank, int W, const int32_t* send_rows, const int32_t* rank_offsets,
+                             int32_t* row_of, uint16_t* send_x, int32_t* send_ids, float* send_w,
+                             chord_stream_t stream) {
+  clear_detail();
+  chord_status_t st = check_ep_args(T, topk, E_rank, W);
+  if (st != CHORD_OK) return st;
+  if (H < 8 || H % 8) return fail(CHORD_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 8", H);
+  if (T == 0) return CHORD_OK;
+  if (!hidden || !topk_ids || !topk_weights || !send_rows || !rank_offsets || !row_of || !send_x || !send_ids || !send_w)
+    return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(send_x)) & 15)
+    return fail(CHORD_ERR_INVALID_ARG, "hidden and send_x must be 16-byte aligned");
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
+  const cudaError_t err = launch_ep_pack(hidden, topk_ids, topk_weights, T, H, topk, E_rank, W, send_rows, rank_offsets,
+                                         send_x, send_ids, send_w, row_of, num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "ep pack launch");
+}
+
+chord_status_t chord_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t T, int H, int W, uint16_t* out,
+                                chord_stream_t stream) {
+  clear_detail();
+  if (T < 0 || W < 1 || W > 64) return fail(CHORD_ERR_INVALID_ARG, "T=%lld W=%d", (long long)T, W);
+  if (H < 8 || H % 8) return fail(CHORD_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 8", H);
+  if (T == 0) return CHORD_OK;
+  if (!row_of || !out) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(back) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(CHORD_ERR_INVALID_ARG, "back and out must be 16-byte aligned");
+  chord_status_t st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
+  const cudaError_t err =
+      launch_ep_combine(back, row_of, T * W, T, H, W, out, num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "ep combine launch");
+}
+
+chord_status_t chord_round_bf16(const float* in, int64_t n, uint16_t* out, chord_stream_t stream) {
+  clear_detail();
+  if (n < 0) return fail(CHORD_ERR_INVALID_ARG, "n=%lld", (long long)n);
+  if (n == 0) return CHORD_OK;
+  if (!in || !out) return fail(CHORD_ERR_INVALID_ARG, "null pointer");
+  chord_status_t st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
+  const cudaError_t err = launch_round_bf16(in, n, out, num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "round launch");
 }
 
 chord_status_t chord_set_timing_events(void* const* events, int n) {

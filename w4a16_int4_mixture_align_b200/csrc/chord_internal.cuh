@@ -415,6 +415,7 @@ struct ForwardArgs {
   uint16_t* xs;    // [cap, H] bf16 hidden rows in sorted order (tensor-core schedule)
   int32_t* slot_pos;  // [T*topk] sorted position of each local flat slot (tensor-core schedule)
   bool y_blocked;     // y is by sorted position in 128-column blocks
+  bool out_f32;       // out receives the FP32 sums (float [T, H]) instead of their BF16 rounding
   bool pdl;           // launch the streaming GEMMs and the combine early (programmatic)
   uint32_t* status;
   uint32_t* stream_flags;   // [2][kMaxStreamWorkers][8] stream-K flags (gate_up, down)
@@ -459,6 +460,17 @@ struct GroupedArgs {
 // The GEMM of the grouped operators: out[row] = x[row] . W[e]^T for every valid row.
 cudaError_t launch_tc_grouped(const GroupedArgs& g, cudaStream_t stream);
 cudaError_t launch_stream_grouped(const GroupedArgs& g, cudaStream_t stream);  // token chunk = g.bm
+
+// Exchange steps of sharded deployments (shard.cu).
+cudaError_t launch_ep_route(const int32_t* topk_ids, int64_t T, int topk, int E_rank, int W, int32_t* ids_tw,
+                            int32_t* row_of, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_pack(const uint16_t* x, const int32_t* topk_ids, const float* topk_weights, int64_t T, int H,
+                           int topk, int E_rank, int W, const int32_t* send_rows, const int32_t* rank_offsets,
+                           uint16_t* send_x, int32_t* send_ids, float* send_w, int32_t* row_of, int num_sms,
+                           cudaStream_t stream);
+cudaError_t launch_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t rows_cap, int64_t T, int H, int W,
+                              uint16_t* out, int num_sms, cudaStream_t stream);
+cudaError_t launch_round_bf16(const float* in, int64_t n, uint16_t* out, int num_sms, cudaStream_t stream);
 
 // Adds n to the process-wide kernel launch counter (chord_launch_count).
 void count_launches(int n);

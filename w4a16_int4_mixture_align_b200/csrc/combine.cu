@@ -22,10 +22,12 @@ constexpr int kCombineCols = kCombineThreads * 8 * kCombineVecs;  // outputs per
 // accumulates its token's local slots in ascending j. BLOCKED selects y by sorted position
 // in 128-column blocks [H/128][cap][128] (tensor-core schedule) instead of y by flat slot
 // [T*topk, H] (streaming schedule).
-template <bool BLOCKED>
+// F32OUT writes the FP32 sums (float [T, H]) instead of their BF16 rounding: the partial
+// output of one tensor-parallel rank, which the ranks add before the single rounding.
+template <bool BLOCKED, bool F32OUT>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const int32_t* __restrict__ topk_ids, const float* __restrict__ topk_weights,
-    const float* __restrict__ y, const int32_t* __restrict__ slot_pos, uint16_t* __restrict__ out, int64_t T,
+    const float* __restrict__ y, const int32_t* __restrict__ slot_pos, void* __restrict__ out_raw, int64_t T,
     int H, int topk, int E, int64_t cap, const int32_t* __restrict__ ntp, int block_m) {
   grid_dep_wait();  // launched early: y comes from the down kernel
   const int lane = threadIdx.x & 31;
@@ -107,6 +109,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     for (int u = 0; u < kCombineVecs; ++u) {
       const int c = c0 + u * kCombineThreads * 8;
       if (c >= H) continue;
+      if (F32OUT) {
+        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(out_raw) + t * H + c);
+        o4[0] = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+        o4[1] = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+        continue;
+      }
+      uint16_t* out = static_cast<uint16_t*>(out_raw);
       uint32_t o[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -152,15 +161,12 @@ cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
   int64_t grid = a.T * ((a.H + kCombineCols - 1) / kCombineCols);
   if (grid > int64_t(a.num_sms) * 64) grid = int64_t(a.num_sms) * 64;
-  cudaError_t err;
-  if (a.y_blocked)
-    err = launch_pdl(a.pdl, combine_kernel<true>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
-                     a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
-                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap, a.ntp, a.block_m);
-  else
-    err = launch_pdl(a.pdl, combine_kernel<false>, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
-                     a.topk_ids, a.topk_weights, static_cast<const float*>(a.y),
-                     static_cast<const int32_t*>(a.slot_pos), a.out, a.T, a.H, a.topk, a.E, a.cap, a.ntp, a.block_m);
+  auto kern = a.y_blocked ? (a.out_f32 ? combine_kernel<true, true> : combine_kernel<true, false>)
+                          : (a.out_f32 ? combine_kernel<false, true> : combine_kernel<false, false>);
+  const cudaError_t err = launch_pdl(a.pdl, kern, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream, a.topk_ids,
+                                     a.topk_weights, static_cast<const float*>(a.y),
+                                     static_cast<const int32_t*>(a.slot_pos), static_cast<void*>(a.out), a.T, a.H,
+                                     a.topk, a.E, a.cap, a.ntp, a.block_m);
   count_launches(1);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
