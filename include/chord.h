@@ -231,7 +231,8 @@ CHORD_API int chord_select_block_m(int64_t T, int topk, int E_local, int E_globa
  *              CHORD_WORKSPACE_HEADER_BYTES hold the device status word (offset 0) and the
  *              flags with which the weight-streaming GEMM's stream-K workers hand partial
  *              sums to one another (each flag is reset by its reader): zero them once after
- *              allocating. The rest is scratch that needs no initialisation.
+ *              allocating, and again after a call that raised CHORD_DEV_TIMEOUT (its
+ *              flags may be left set). The rest is scratch that needs no initialisation.
  *
  * Requires H % 128 == 0, I % 128 == 0, 1 <= block_m <= 256 (same as used for align).
  * Concurrent forwards must not share a workspace.

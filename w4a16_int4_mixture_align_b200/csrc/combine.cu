@@ -13,19 +13,57 @@ namespace chord {
 namespace {
 
 constexpr int kCombineThreads = 128;
-constexpr int kCombineVecs = 2;                    // 8-output vectors per thread and item
-constexpr int kCombineCols = kCombineThreads * 8 * kCombineVecs;  // outputs per work item
+constexpr int kCombineVecs = 4;                    // 8-output vectors per lane and unit
+constexpr int kUnitCols = 32 * 8 * kCombineVecs;   // outputs per unit (one warp)
+constexpr int kSlotGroup = 2;                      // local slots whose rows are loaded together
 
-// Work item = (token t, 2048 consecutive outputs); a thread owns two vectors of 8 outputs,
-// 1024 apart, so each slot's loads come in independent pairs. Lane j % 32
-// of every warp holds slot j's weight and row of y (top-k up to 64), and each output
-// accumulates its token's local slots in ascending j. BLOCKED selects y by sorted position
-// in 128-column blocks [H/128][cap][128] (tensor-core schedule) instead of y by flat slot
-// [T*topk, H] (streaming schedule).
-// F32OUT writes the FP32 sums (float [T, H]) instead of their BF16 rounding: the partial
-// output of one tensor-parallel rank, which the ranks add before the single rounding.
+// A token's slots as one warp sees them: lane j % 32 of half j / 32 holds slot j's row
+// of y (-1 when the slot is not local or its position is unknown) and top-k weight.
+struct SlotRows {
+  int row[2];  // < 2^31: the routing capacity and T*topk are checked below that
+  float w[2];
+};
+
+// Issues every load of token t's slot metadata at once (ids, weights and positions do
+// not depend on one another), so a prefetch of the next unit's token overlaps the current
+// unit's rows of y.
+template <bool BLOCKED>
+__device__ __forceinline__ void load_slot_rows(SlotRows& m, int64_t t, int lane, const int32_t* __restrict__ topk_ids,
+                                               const float* __restrict__ topk_weights,
+                                               const int32_t* __restrict__ slot_pos, int topk, int E, int64_t cap,
+                                               bool routed) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int j = h * 32 + lane;
+    m.row[h] = -1;
+    m.w[h] = 0.f;
+    if (j < topk) {
+      const int64_t f = t * topk + j;
+      const int e = __ldg(topk_ids + f);
+      const float w = __ldg(topk_weights + f);
+      const int pos = BLOCKED ? __ldg(slot_pos + f) : 0;
+      if (routed && unsigned(e) < unsigned(E)) {
+        m.w[h] = w;
+        m.row[h] = BLOCKED ? ((pos >= 0 && pos < cap) ? pos : -1) : int(f);
+      }
+    }
+  }
+}
+
+// Unit = (token t, kUnitCols consecutive outputs), one warp; a lane owns kCombineVecs
+// vectors of 8 outputs, 256 apart, so a warp's loads and stores of one vector index are
+// contiguous. The token's local slots are found with one ballot and taken in ascending j,
+// kSlotGroup at a time: the group's rows are all requested before any is summed, and slots
+// that are not local cost nothing. Each output accumulates w_j * y_j in ascending j in
+// FP32 (product rounded, then added). Warps walk units with a grid stride and load the
+// next unit's slot metadata before summing the current one, so a unit costs one memory
+// round trip per slot group.
+// BLOCKED selects y by sorted position in 128-column blocks [H/128][cap][128] (tensor-core
+// schedule) instead of y by flat slot [T*topk, H] (streaming schedule). F32OUT writes the
+// FP32 sums (float [T, H]) instead of their BF16 rounding: the partial output of one
+// tensor-parallel rank, which the ranks add before the single rounding.
 template <bool BLOCKED, bool F32OUT>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+__global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(
     const int32_t* __restrict__ topk_ids, const float* __restrict__ topk_weights,
     const float* __restrict__ y, const int32_t* __restrict__ slot_pos, void* __restrict__ out_raw, int64_t T,
     int H, int topk, int E, int64_t cap, const int32_t* __restrict__ ntp, int block_m) {
@@ -34,61 +72,59 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
   // routing built for another block_m: the GEMMs computed nothing, so every row is zero
   // (the GEMM kernels raise CHORD_DEV_BLOCK_M_MISMATCH)
   const bool routed = ntp[1] == routing_tag(block_m);
-  const int nchunk = (H + kCombineCols - 1) / kCombineCols;
-  for (int64_t item = blockIdx.x; item < T * nchunk; item += gridDim.x) {
-    const int64_t t = item / nchunk;
-    const int c0 = int(item % nchunk) * kCombineCols + threadIdx.x * 8;
-    // slot j's row of y (lane j % 32 of set j / 32), or -1 when the slot is not local (or
-    // its position is unknown)
-    int64_t row[2] = {-1, -1};
-    float w[2] = {0.f, 0.f};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = h * 32 + lane;
-      if (j < topk) {
-        const int64_t f = t * topk + j;
-        const int e = __ldg(topk_ids + f);
-        if (routed && unsigned(e) < unsigned(E)) {
-          w[h] = __ldg(topk_weights + f);
-          if (BLOCKED) {
-            const int pos = __ldg(slot_pos + f);
-            row[h] = (pos >= 0 && pos < cap) ? pos : -1;
-          } else {
-            row[h] = f;
-          }
-        }
-      }
-    }
+  const int nseg = (H + kUnitCols - 1) / kUnitCols;
+  const int64_t units = T * nseg;
+  const int64_t nwarps = (int64_t(gridDim.x) * kCombineThreads) >> 5;
+  int64_t u = (int64_t(blockIdx.x) * kCombineThreads + threadIdx.x) >> 5;
+  if (u >= units) return;
+  SlotRows cur;
+  int64_t t = u / nseg;
+  load_slot_rows<BLOCKED>(cur, t, lane, topk_ids, topk_weights, slot_pos, topk, E, cap, routed);
+  for (; u < units; u += nwarps) {
+    const int seg = int(u - t * nseg);
+    // the next unit's token: its metadata loads go out now
+    const int64_t un = u + nwarps;
+    const int64_t tn = un < units ? un / nseg : t;
+    SlotRows nxt = cur;
+    if (tn != t) load_slot_rows<BLOCKED>(nxt, tn, lane, topk_ids, topk_weights, slot_pos, topk, E, cap, routed);
+
+    const int c0 = seg * kUnitCols + lane * 8;
     float acc[kCombineVecs][8];
 #pragma unroll
-    for (int u = 0; u < kCombineVecs; ++u)
+    for (int k = 0; k < kCombineVecs; ++k)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-    // slots in groups of kSlotGroup: the group's rows are all requested before any is
-    // summed (one memory round trip per group, not per slot), then added in ascending j
-    constexpr int kSlotGroup = 4;
-    for (int j0 = 0; j0 < topk; j0 += kSlotGroup) {
-      int64_t rj[kSlotGroup];
+      for (int i = 0; i < 8; ++i) acc[k][i] = 0.f;
+    // local slots, ascending j (warp-uniform masks)
+    uint32_t mask0 = __ballot_sync(0xffffffffu, cur.row[0] >= 0);
+    uint32_t mask1 = topk > 32 ? __ballot_sync(0xffffffffu, cur.row[1] >= 0) : 0u;
+    while (mask0 | mask1) {
+      int rj[kSlotGroup];
       float wj[kSlotGroup];
       float4 v[kSlotGroup][kCombineVecs][2];
 #pragma unroll
       for (int q = 0; q < kSlotGroup; ++q) {
-        const int j = j0 + q;
         rj[q] = -1;
         wj[q] = 0.f;
-        if (j < topk) {
-          rj[q] = __shfl_sync(0xffffffffu, j < 32 ? row[0] : row[1], j & 31);
-          wj[q] = __shfl_sync(0xffffffffu, j < 32 ? w[0] : w[1], j & 31);
+        if (mask0) {
+          const int src = __ffs(mask0) - 1;
+          mask0 &= mask0 - 1;
+          rj[q] = __shfl_sync(0xffffffffu, cur.row[0], src);
+          wj[q] = __shfl_sync(0xffffffffu, cur.w[0], src);
+        } else if (mask1) {
+          const int src = __ffs(mask1) - 1;
+          mask1 &= mask1 - 1;
+          rj[q] = __shfl_sync(0xffffffffu, cur.row[1], src);
+          wj[q] = __shfl_sync(0xffffffffu, cur.w[1], src);
         }
 #pragma unroll
-        for (int u = 0; u < kCombineVecs; ++u) {
-          const int c = c0 + u * kCombineThreads * 8;
-          v[q][u][0] = v[q][u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < kCombineVecs; ++k) {
+          const int c = c0 + k * 256;
+          v[q][k][0] = v[q][k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (rj[q] >= 0 && c < H) {
             const float* src =
-                BLOCKED ? y + ((int64_t(c >> 7) * cap + rj[q]) << 7) + (c & 127) : y + rj[q] * H + c;
-            v[q][u][0] = __ldcs(reinterpret_cast<const float4*>(src));
-            v[q][u][1] = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+                BLOCKED ? y + ((int64_t(c >> 7) * cap + rj[q]) << 7) + (c & 127) : y + int64_t(rj[q]) * H + c;
+            v[q][k][0] = __ldcs(reinterpret_cast<const float4*>(src));
+            v[q][k][1] = __ldcs(reinterpret_cast<const float4*>(src) + 1);
           }
         }
       }
@@ -97,32 +133,34 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
       for (int q = 0; q < kSlotGroup; ++q) {
         if (rj[q] < 0) continue;
 #pragma unroll
-        for (int u = 0; u < kCombineVecs; ++u) {
-          const float vv[8] = {v[q][u][0].x, v[q][u][0].y, v[q][u][0].z, v[q][u][0].w,
-                               v[q][u][1].x, v[q][u][1].y, v[q][u][1].z, v[q][u][1].w};
+        for (int k = 0; k < kCombineVecs; ++k) {
+          const float vv[8] = {v[q][k][0].x, v[q][k][0].y, v[q][k][0].z, v[q][k][0].w,
+                               v[q][k][1].x, v[q][k][1].y, v[q][k][1].z, v[q][k][1].w};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(wj[q], vv[i]));
+          for (int i = 0; i < 8; ++i) acc[k][i] = __fadd_rn(acc[k][i], __fmul_rn(wj[q], vv[i]));
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < kCombineVecs; ++u) {
-      const int c = c0 + u * kCombineThreads * 8;
+    for (int k = 0; k < kCombineVecs; ++k) {
+      const int c = c0 + k * 256;
       if (c >= H) continue;
       if (F32OUT) {
         float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(out_raw) + t * H + c);
-        o4[0] = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
-        o4[1] = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+        o4[0] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+        o4[1] = make_float4(acc[k][4], acc[k][5], acc[k][6], acc[k][7]);
         continue;
       }
       uint16_t* out = static_cast<uint16_t*>(out_raw);
       uint32_t o[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        o[i] = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[u][2 * i]))) |
-               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[u][2 * i + 1]))) << 16);
+        o[i] = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[k][2 * i]))) |
+               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc[k][2 * i + 1]))) << 16);
       *reinterpret_cast<uint4*>(out + t * H + c) = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    cur = nxt;
+    t = tn;
   }
 }
 
@@ -159,8 +197,11 @@ __global__ void validate_kernel(const int32_t* __restrict__ topk_ids,
 
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
-  int64_t grid = a.T * ((a.H + kCombineCols - 1) / kCombineCols);
-  if (grid > int64_t(a.num_sms) * 64) grid = int64_t(a.num_sms) * 64;
+  // one unit per warp, warps resident all at once (4 CTAs per SM by the launch bounds):
+  // each walks its units with the next unit's metadata in flight
+  const int64_t units = a.T * ((a.H + kUnitCols - 1) / kUnitCols);
+  int64_t grid = (units + kCombineThreads / 32 - 1) / (kCombineThreads / 32);
+  if (grid > int64_t(a.num_sms) * 4) grid = int64_t(a.num_sms) * 4;
   auto kern = a.y_blocked ? (a.out_f32 ? combine_kernel<true, true> : combine_kernel<true, false>)
                           : (a.out_f32 ? combine_kernel<false, true> : combine_kernel<false, false>);
   const cudaError_t err = launch_pdl(a.pdl, kern, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream, a.topk_ids,
