@@ -36,7 +36,6 @@ __host__ __device__ inline int multi_chunk(int64_t n, int E) {
   const int64_t g = (n + kChunkSmall - 1) / kChunkSmall;
   return int64_t(E) * g <= kMaxHistEntries ? kChunkSmall : kChunk;
 }
-constexpr int kMaxE = 1024;
 // Up to this many 1024-slot chunks the routing sort runs in one CTA (one launch); above
 // it the count / scan / scatter kernels spread the slots over the GPU (one CTA sorting
 // 32 chunks took ~70 us).
@@ -233,7 +232,6 @@ __global__ void __launch_bounds__(1024) align_single_kernel(
 // best unselected slot; every round the warp takes the largest of them (larger value,
 // or the lower id on equal values), and only the lane that supplied it rescans. Lane
 // r % 32 ends with the expert of rank r (descending logit, ties to the lower id).
-constexpr int kRouterMaxG = 1024;
 constexpr int kNoExpert = 0x7fffffff;
 
 template <int PER>
@@ -353,7 +351,7 @@ __global__ void __launch_bounds__(1024) router_align_single_kernel(
 
 
 // ---- multi CTA ---------------------------------------------------------------------
-// workspace: chunk_hist [E][G] int32 | cnt [E] | off [E+1]
+// workspace: chunk_hist [E][G] int32 | cnt [E]
 constexpr int kWarpsPerCta = 4;
 
 __global__ void __launch_bounds__(32 * kWarpsPerCta) align_count_kernel(
@@ -371,84 +369,107 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) align_count_kernel(
   for (int e = lane; e < E; e += 32) chunk_hist[int64_t(e) * G + chunk] = row[e];
 }
 
-__global__ void __launch_bounds__(1024) align_scan_kernel(int E, int block_m, int64_t G,
-                                                          int* __restrict__ chunk_hist,
-                                                          int* __restrict__ cnt_g,
-                                                          int* __restrict__ off_g,
-                                                          int32_t* __restrict__ ntp_out,
-                                                          int32_t* __restrict__ offsets_out) {
-  __shared__ int off[kMaxE + 1];
-  __shared__ int wsum[33];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // a warp per expert: exclusive prefix of its chunk counts over windows of 32 x R chunks,
-  // each lane loading its R consecutive counts at once (one round trip per window)
+// A warp per expert (32 experts per CTA): the exclusive prefix of the expert's run counts,
+// in place, over windows of 32 x R runs (each lane loads its R consecutive counts at
+// once: one round trip per window), and the expert's total. The experts' offsets are
+// scanned by every scatter CTA itself, so no single CTA walks all experts.
+__global__ void __launch_bounds__(1024) align_scan_kernel(int E, int64_t G, int* __restrict__ chunk_hist,
+                                                          int* __restrict__ cnt_g) {
+  const int lane = threadIdx.x & 31;
+  const int e = int(blockIdx.x) * 32 + (threadIdx.x >> 5);
+  if (e >= E) return;
   constexpr int R = 8;
-  for (int e = warp; e < E; e += int(blockDim.x >> 5)) {
-    int* h = chunk_hist + int64_t(e) * G;
-    int run = 0;
-    for (int64_t base = 0; base < G; base += 32 * R) {
-      int c[R];
+  int* h = chunk_hist + int64_t(e) * G;
+  int run = 0;
+  for (int64_t base = 0; base < G; base += 32 * R) {
+    int c[R];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int64_t g = base + lane * R + i;
-        c[i] = g < G ? h[g] : 0;
-      }
-      int lsum = 0;
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int x = c[i];
-        c[i] = lsum;
-        lsum += x;
-      }
-      int incl = lsum;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
-      }
-      const int excl = run + incl - lsum;
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int64_t g = base + lane * R + i;
-        if (g < G) h[g] = excl + c[i];
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
+    for (int i = 0; i < R; ++i) {
+      const int64_t g = base + lane * R + i;
+      c[i] = g < G ? h[g] : 0;
     }
-    if (lane == 0) {
-      cnt_g[e] = run;
-      off[e] = (run + block_m - 1) / block_m * block_m;
+    int lsum = 0;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int x = c[i];
+      c[i] = lsum;
+      lsum += x;
     }
+    int incl = lsum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    const int excl = run + incl - lsum;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int64_t g = base + lane * R + i;
+      if (g < G) h[g] = excl + c[i];
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
+  if (lane == 0) cnt_g[e] = run;
+}
+
+// Exclusive prefix of vals[0, count) in place for any count (each thread sums a run of
+// consecutive values, the runs' sums are scanned across the block); returns the total.
+// tmp holds blockDim.x ints, warp_sums 33.
+__device__ int block_exclusive_scan_runs(int* vals, int count, int* tmp, int* warp_sums) {
+  const int tid = threadIdx.x;
+  const int per = (count + int(blockDim.x) - 1) / int(blockDim.x);
+  const int b = tid * per;
+  int sum = 0;
+  for (int i = 0; i < per; ++i)
+    if (b + i < count) sum += vals[b + i];
+  tmp[tid] = sum;
   __syncthreads();
-  const int total = block_exclusive_scan(off, E, wsum);
-  for (int e = tid; e < E; e += blockDim.x) off_g[e] = off[e];
-  if (tid == 0) {
-    off_g[E] = total;
-    ntp_out[0] = total;
-    ntp_out[1] = routing_tag(block_m);
-  }
-  if (offsets_out) {
-    for (int e = tid; e < E; e += blockDim.x) offsets_out[e] = off[e];
-    if (tid == 0) offsets_out[E] = total;
-  }
+  const int total = block_exclusive_scan(tmp, int(blockDim.x), warp_sums);
+  int run = tmp[tid];
+  for (int i = 0; i < per; ++i)
+    if (b + i < count) {
+      const int x = vals[b + i];
+      vals[b + i] = run;
+      run += x;
+    }
+  __syncthreads();
+  return total;
 }
 
 __global__ void __launch_bounds__(32 * kWarpsPerCta) align_scatter_kernel(
     const int32_t* __restrict__ ids, int64_t n, int E, int block_m, int64_t G, int64_t cap,
     int64_t nblocks, int csz, const int* __restrict__ chunk_hist, const int* __restrict__ cnt_g,
-    const int* __restrict__ off_g, int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids) {
+    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntp_out,
+    int32_t* __restrict__ offsets_out) {
   extern __shared__ int smem[];
+  __shared__ int wsum[33];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* row = smem + warp * E;
+  // the experts' padded offsets, scanned by this CTA: off[e] (E + 1 entries)
+  int* off = smem + kWarpsPerCta * E;
+  int* tmp = off + E + 1;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) off[e] = (cnt_g[e] + block_m - 1) / block_m * block_m;
+  __syncthreads();
+  const int total = block_exclusive_scan_runs(off, E, tmp, wsum);
+  if (threadIdx.x == 0) off[E] = total;
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0) {
+      ntp_out[0] = total;
+      ntp_out[1] = routing_tag(block_m);
+    }
+    if (offsets_out)
+      for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets_out[e] = off[e];
+  }
   const int64_t chunk = int64_t(blockIdx.x) * kWarpsPerCta + warp;
   if (chunk < G) {
-    for (int e = lane; e < E; e += 32) row[e] = off_g[e] + chunk_hist[int64_t(e) * G + chunk];
+    for (int e = lane; e < E; e += 32) row[e] = off[e] + chunk_hist[int64_t(e) * G + chunk];
     __syncwarp();
     int v[kSteps];
     load_steps(ids, n, chunk * csz, csz / 32, v);
     chunk_scatter(v, csz / 32, chunk * csz, E, key_bits(E), row, sorted_ids);
   }
-  fill_tail(cnt_g, off_g, E, block_m, n, cap, nblocks, sorted_ids, expert_ids,
+  fill_tail(cnt_g, off, E, block_m, n, cap, nblocks, sorted_ids, expert_ids,
             int64_t(blockIdx.x) * blockDim.x + threadIdx.x, int64_t(gridDim.x) * blockDim.x);
 }
 
@@ -458,7 +479,7 @@ size_t align_workspace_bytes(int64_t n, int E) {
   if ((n + kChunk - 1) / kChunk <= kSingleMaxChunks) return 0;
   const int csz = multi_chunk(n, E);
   const int64_t G = (n + csz - 1) / csz;
-  return align256(uint64_t(E) * G * 4) + align256(uint64_t(E) * 4) + align256(uint64_t(E + 1) * 4);
+  return align256(uint64_t(E) * G * 4) + align256(uint64_t(E) * 4);
 }
 
 cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int64_t cap,
@@ -479,19 +500,20 @@ cudaError_t launch_align(const int32_t* ids, int64_t n, int E, int block_m, int6
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* chunk_hist = reinterpret_cast<int*>(ws);
   int* cnt = reinterpret_cast<int*>(ws + align256(uint64_t(E) * G * 4));
-  int* off = reinterpret_cast<int*>(ws + align256(uint64_t(E) * G * 4) + align256(uint64_t(E) * 4));
   const int64_t ctas = (G + kWarpsPerCta - 1) / kWarpsPerCta;
   const size_t smem = size_t(kWarpsPerCta) * E * sizeof(int);
+  // scatter: the warps' rows, then the experts' offsets (E + 1) and the scan's run sums
+  const size_t smem_scatter = smem + (size_t(E) + 1 + 32 * kWarpsPerCta) * sizeof(int);
   cudaError_t err = cudaFuncSetAttribute(align_count_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
+                             int(smem_scatter));
   if (err != cudaSuccess) return err;
   align_count_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem, stream>>>(ids, n, E, G, csz, chunk_hist);
-  align_scan_kernel<<<1, 1024, 0, stream>>>(E, block_m, G, chunk_hist, cnt, off, ntp, offsets);
-  align_scatter_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem, stream>>>(
-      ids, n, E, block_m, G, cap, nblocks, csz, chunk_hist, cnt, off, sorted_ids, expert_ids);
+  align_scan_kernel<<<unsigned((E + 31) / 32), 1024, 0, stream>>>(E, G, chunk_hist, cnt);
+  align_scatter_kernel<<<unsigned(ctas), 32 * kWarpsPerCta, smem_scatter, stream>>>(
+      ids, n, E, block_m, G, cap, nblocks, csz, chunk_hist, cnt, sorted_ids, expert_ids, ntp, offsets);
   count_launches(3);
   return cudaGetLastError();
 }
