@@ -26,6 +26,12 @@ The grouped_* workloads time the grouped operators instead (one step = one
 chord_grouped_contiguous / chord_grouped_masked call: routing pass + GEMM) on an EP8 shard
 (48 experts) at the rows per expert the blog's grouped table uses.
 
+The exchange workloads time the device steps around a sharded layer on one GPU (the
+collectives between them need several): ep8_exchange_decode / _prefill = chord_ep_plan +
+chord_ep_pack + chord_ep_combine for the EP8 decode (128 tokens) or prefill (8192 tokens)
+batch of one rank over 8 ranks (the returned rows synthetic), and tp8_reduce =
+chord_round_bf16 of the TP8 prefill partial sums.
+
 --impl reference times the CPU oracle (test infrastructure) on the headline workload on
 the host cores: rank 0 only, other ranks exit without work.
 """
@@ -56,6 +62,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 EV_EVERY = 8  # steps per step that records the per-kernel timing events
 DEFAULT_STEPS = {"ep8_decode": 2000, "tp8_decode": 2000, "tiny": 2000, "ep8_prefill": 200,
                  "tp8_prefill": 400, "skew": 100}
+EXCHANGE_WORKLOADS = ("ep8_exchange_decode", "ep8_exchange_prefill", "tp8_reduce")
 
 
 def describe(cfg: inputs.MoEConfig) -> str:
@@ -639,6 +646,7 @@ def run_grouped(args, rank, world, local_rank):
         return None
 
     hbm, tf_burst, tf_sust, pk_kind = peaks()
+    clocks = sampler.summary(t_wall0, t_wall1)
     gemm_us = seg_ms[1] * 1000.0
     # the library's default schedule: expected rows per expert (masked: the expected_m hint;
     # contiguous: padded rows / E) above 16 go to the tensor cores
@@ -648,10 +656,10 @@ def run_grouped(args, rank, world, local_rank):
             else (8 if expected <= 8 else (16 if expected <= 16 else 32)))
     if tensor:
         achieved = work["flops"] / (gemm_us * 1e-6) / 1e12
+        tf_peak, tf_src = tensor_peak(clocks, tf_burst, tf_sust, pk_kind)
         roofline = {"bound": "tensor", "kernel": "tc_gemm (plain epilogue)", "achieved": round(achieved, 1),
-                    "peak": tf_sust, "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
-                    "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long run of calls)",
-                    "peak_burst": tf_burst, "frac_of_burst": round(achieved / tf_burst, 4),
+                    "peak": tf_peak, "unit": "TFLOP/s", "frac": round(achieved / tf_peak, 4), "peak_source": tf_src,
+                    "frac_of_burst": round(achieved / tf_burst, 4), "frac_of_sustained": round(achieved / tf_sust, 4),
                     "traffic": recorded_traffic("tc_gemm_plain", args.workload),
                     "algorithmic_flops_per_launch": work["flops"]}
     else:
@@ -674,7 +682,7 @@ def run_grouped(args, rank, world, local_rank):
         "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": x_h.numel() * 2 + r_h.numel() * 4, "d2h_bytes_per_step": out_h[0].numel() * 2},
         "gpu_launches": int(launches),
-        "clocks": sampler.summary(t_wall0, t_wall1),
+        "clocks": clocks,
     }
 
 
@@ -755,6 +763,9 @@ def cpu_baseline(cfg, max_seconds=30.0):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    if args.workload in EXCHANGE_WORKLOADS:
+        return {"impl": "reference", "unavailable": "the oracle has no exchange steps: they only move rows "
+                "(bit-exact against their definitions in the tests)"}
     import oracle
     oracle.build()
     if args.workload in inputs.GROUPED_CONFIGS:
@@ -802,13 +813,179 @@ def run_reference_grouped(args, world):
 
 # ------------------------------------------------------------------------------ main
 
+def run_exchange(args, rank, world, local_rank):
+    """The device steps of a sharded layer's exchange on one GPU (the collectives between
+    them need several GPUs and are not timed here).
+
+    ep8_exchange_decode / _prefill: the EP8 decode (128 tokens) or prefill (8192 tokens)
+    batch of one rank, top-8 of 384 experts by global id, over 8 expert-parallel ranks of
+    48 experts: chord_ep_plan (send rows by destination rank),
+    chord_ep_pack (hidden rows, local ids and weights of every send row) and
+    chord_ep_combine (the returned rows summed per token in rank order; synthetic rows
+    stand in for what the other ranks send back). tp8_reduce: chord_round_bf16 of one
+    TP8 prefill output, FP32 [4096, 7168], after the all-reduce."""
+    import torch
+    from w4a16_int4_mixture_align_b200 import chord
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    K, W = args.steps, args.warmup
+    if args.workload.startswith("ep8_exchange"):
+        cfg = inputs.CONFIGS["ep8_decode" if args.workload.endswith("decode") else "ep8_prefill"]
+        rcfg = inputs.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})
+        ids_np, tw_np = inputs.make_routing(rcfg, global_ids=True)
+        x_np = inputs.make_hidden(rcfg)
+        T, H, k, E_rank, Wr = cfg.T, cfg.H, cfg.topk, cfg.E, cfg.E_global // cfg.E
+        host_in = [torch.from_numpy(x_np.view(np.int16)), torch.from_numpy(ids_np), torch.from_numpy(tw_np)]
+        send_rows = torch.empty(T * Wr, dtype=torch.int32, device=dev)
+        offsets = torch.empty(Wr + 1, dtype=torch.int32, device=dev)
+        row_of = torch.empty(T * Wr, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(chord.chord_ep_plan_workspace_bytes(T, Wr), 256), dtype=torch.uint8, device=dev)
+        send_x = torch.empty((T * Wr, H), dtype=torch.bfloat16, device=dev)
+        send_ids = torch.empty((T * Wr, k), dtype=torch.int32, device=dev)
+        send_w = torch.empty((T * Wr, k), dtype=torch.float32, device=dev)
+        # the rows the other ranks return: one per send row (counted on the host)
+        n_send = sum(1 for t in range(T) for d in range(Wr)
+                     if np.any((ids_np[t] >= d * E_rank) & (ids_np[t] < (d + 1) * E_rank)))
+        back = torch.from_numpy(np.random.default_rng(rank).standard_normal((max(n_send, 1), H)).astype(np.float32))
+        back = back.to(dev).to(torch.bfloat16)
+        out_shape, out_dtype = (T, H), torch.bfloat16
+
+        def steps(xin, oo):
+            xx, ii, ww = xin
+            xx = xx.view(torch.bfloat16)
+            return [lambda: chord.chord_ep_plan(ii, E_rank, Wr, send_rows, offsets, row_of, ws),
+                    lambda: chord.chord_ep_pack(xx, ii, ww, E_rank, Wr, send_rows, offsets, row_of, send_x, send_ids,
+                                                send_w),
+                    lambda: chord.chord_ep_combine(back, row_of, Wr, oo)]
+        names = ["plan", "pack", "combine"]
+        # algorithmic bytes: plan reads the ids and writes the send rows and row_of; pack
+        # reads each hidden row once (a row sent to several ranks is read again from L2)
+        # and writes every send row (+ its ids and weights); combine reads the returned rows
+        # and writes out
+        nbytes = [T * k * 4 + 2 * T * Wr * 4 + (Wr + 1) * 4,
+                  T * H * 2 + n_send * H * 2 + n_send * k * 8 + n_send * 4 + T * Wr * 4,
+                  n_send * H * 2 + T * Wr * 4 + T * H * 2]
+        desc = (f"{args.workload}: EP8 batch T={T} top-{k} (global ids) over {Wr} ranks x {E_rank} experts, "
+                f"H={H}: {n_send} send rows; plan + pack + combine (the all-to-all legs not included)")
+    else:
+        cfg = inputs.CONFIGS["tp8_prefill"]
+        T, H = cfg.T, cfg.H
+        host_in = [torch.from_numpy(np.random.default_rng(rank).standard_normal((T, H)).astype(np.float32))]
+        out_shape, out_dtype = (T, H), torch.bfloat16
+
+        def steps(xin, oo):
+            return [lambda: chord.chord_round_bf16(xin[0], oo)]
+        names = ["round"]
+        nbytes = [T * H * 4 + T * H * 2]
+        desc = f"tp8_reduce: chord_round_bf16 of a TP8 prefill output, FP32 [{T}, {H}] -> BF16 (after the all-reduce)"
+
+    dev_in = [t.to(dev) for t in host_in]
+    out = torch.empty(out_shape, dtype=out_dtype, device=dev)
+    fns = steps(dev_in, out)
+
+    def step():
+        for f in fns:
+            f()
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    # timed: one graph replay of the K steps; per kernel: a second graph with events between
+    launches0 = chord.chord_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(K):
+            step()
+    launches = chord.chord_launch_count() - launches0
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(fns) + 1)] for _ in range(K)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        for kk in range(K):
+            ev[kk][0].record(stream)
+            for i, f in enumerate(fns):
+                f()
+                ev[kk][i + 1].record(stream)
+    graph.replay()
+    g2.replay()
+    torch.cuda.synchronize()
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    graph.replay()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    elapsed_ms = start.elapsed_time(stop)
+    g2.replay()
+    torch.cuda.synchronize()
+    seg_ms = np.array([[ev[kk][i].elapsed_time(ev[kk][i + 1]) for i in range(len(fns))] for kk in range(K)]).mean(0)
+    del graph, g2
+
+    # end to end: the inputs from pinned host memory, the output back, two buffer slots
+    host_pin = [t.pin_memory() for t in host_in]
+    din = [[torch.empty_like(t) for t in dev_in] for _ in range(2)]
+    outd = [torch.empty_like(out) for _ in range(2)]
+    out_h = [torch.empty(out_shape, dtype=torch.int16).pin_memory() for _ in range(2)]
+    slot_fns = [steps(din[s], outd[s]) for s in range(2)]
+
+    def copy_in(s):
+        for dst, src in zip(din[s], host_pin):
+            dst.copy_(src, non_blocking=True)
+
+    def compute(s):
+        for f in slot_fns[s]:
+            f()
+
+    def copy_out(s):
+        out_h[s].copy_(outd[s].view(torch.int16), non_blocking=True)
+
+    e2e_ms = pipelined_e2e_ms(K, W, copy_in, compute, copy_out, stream, dev, world)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    stats = max_over_ranks([elapsed_ms, e2e_ms, *seg_ms.tolist()], world, device=dev)
+    elapsed_ms, e2e_ms, seg_ms = stats[0], stats[1], np.array(stats[2:])
+    if rank != 0:
+        return None
+    hbm = peaks()[0]
+    top = int(np.argmax(nbytes))  # the kernel that moves the most bytes
+    achieved = nbytes[top] / (seg_ms[top] * 1e-3) / 1e9
+    return {
+        "metric": "exchange steps of a sharded layer, µs/call; HBM GB/s vs roofline",
+        "value": round(job_us_per_call(elapsed_ms, K, world), 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(elapsed_ms / K, 5), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": desc, "l2": "no flush (each step rewrites its outputs)",
+                   "parallelism": f"replicas x{world}"},
+        "kernels_us": {n: round(v * 1000, 2) for n, v in zip(names, seg_ms)},
+        "roofline": {"bound": "hbm", "kernel": names[top], "achieved": round(achieved, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": int(nbytes[top])},
+        "e2e": {"value": round(job_us_per_call(e2e_ms, K, world), 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_in)),
+                "d2h_bytes_per_step": int(out.numel() * 2)},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["chord", "reference"], default="chord")
-    ap.add_argument("--workload", choices=["all"] + list(inputs.CONFIGS) + sorted(inputs.GROUPED_CONFIGS),
+    ap.add_argument("--workload", choices=["all"] + list(inputs.CONFIGS) + sorted(inputs.GROUPED_CONFIGS)
+                    + list(EXCHANGE_WORKLOADS),
                     default="all",
                     help="all (default): the EP8 decode headline plus every layer workload of the metric")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -817,7 +994,8 @@ def main():
     ap.add_argument("--expected-m", type=int, default=None,
                     help="grouped masked workloads: the expected_m hint (default: the rows per expert)")
     args = ap.parse_args()
-    if args.steps is None and (args.impl == "reference" or args.workload in inputs.GROUPED_CONFIGS):
+    if args.steps is None and (args.impl == "reference" or args.workload in inputs.GROUPED_CONFIGS
+                               or args.workload in EXCHANGE_WORKLOADS):
         args.steps = 3 if args.impl == "reference" else 200
     args.warmup = max(args.warmup, 3)
 
@@ -839,9 +1017,12 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
 
     grouped = args.workload in inputs.GROUPED_CONFIGS
-    line = (run_grouped if grouped else run_chord)(args, rank, world, local_rank)
+    exchange = args.workload in EXCHANGE_WORKLOADS
+    line = (run_exchange if exchange else run_grouped if grouped else run_chord)(args, rank, world, local_rank)
     if line is not None:
-        if world == 1 and not args.no_cpu_baseline:
+        if exchange:
+            line["cpu_baseline"] = None
+        elif world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = (grouped_cpu_baseline(inputs.GROUPED_CONFIGS[args.workload]) if grouped
                                     else cpu_baseline(inputs.CONFIGS[HEADLINE if args.workload == "all"
                                                                          else args.workload]))

@@ -11,7 +11,9 @@
 //      received row, and the source sums a token's returned rows.
 //        chord_ep_plan    send rows grouped by destination rank, ascending token inside
 //                         each (the routing sort of the layer over W "experts" = ranks)
-//        chord_ep_pack    the send buffers: hidden rows, local ids, weights
+//        chord_ep_pack    row_of (the inverse of send_rows), then the send buffers token by
+//                         token: each piece of a hidden row read once and stored into each
+//                         of its send rows, with the local ids and weights
 //        chord_ep_combine out[t] = bf16( sum over ranks d, ascending, of float(back row) )
 //  TP: each rank owns a slice of the intermediate dimension of every expert; its layer
 //      output is a partial sum of the full layer's FP32 result. chord_moe_forward with
@@ -43,35 +45,76 @@ __global__ void __launch_bounds__(256) ep_route_kernel(const int32_t* __restrict
   }
 }
 
-// One warp per send row i < num_rows: the token's hidden row, its slots made local to the
-// destination rank, and row_of[t * W + d] = i for the combine.
-__global__ void __launch_bounds__(256) ep_pack_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_ids,
-                                                      const float* __restrict__ topk_weights, int64_t T, int H, int topk,
-                                                      int E_rank, int W, const int32_t* __restrict__ send_rows,
-                                                      const int32_t* __restrict__ rank_offsets,
-                                                      uint16_t* __restrict__ send_x, int32_t* __restrict__ send_ids,
-                                                      float* __restrict__ send_w, int32_t* __restrict__ row_of) {
-  const int lane = threadIdx.x & 31;
+// row_of[send_rows[i]] = i for every send row i < rank_offsets[W] (the other entries stay
+// -1 from the route kernel): the send row of each (token, rank) pair.
+__global__ void __launch_bounds__(256) ep_invert_kernel(const int32_t* __restrict__ send_rows,
+                                                        const int32_t* __restrict__ rank_offsets, int64_t T, int W,
+                                                        int32_t* __restrict__ row_of) {
   int64_t rows = rank_offsets[W];
   if (rows < 0) rows = 0;
   if (rows > T * W) rows = T * W;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < rows; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t f = send_rows[i];
+    if (f >= 0 && f < T * W) row_of[f] = int32_t(i);
+  }
+}
+
+// One warp per (token t, 1024-column chunk), token-major: the token's send rows
+// (row_of[t*W + d], lane d % 32 of half d / 32) are found with a ballot; each 16-byte vector
+// of the chunk is read once (four per lane) and stored into every one of them, so a row
+// sent to several ranks is read from memory once, and a small batch still spreads over
+// many warps. The chunk-0 warp also writes each send row's slots made local to its rank
+// (-1 elsewhere) and their weights (0 elsewhere).
+constexpr int kPackVecs = 4;                    // 16-byte vectors per lane and chunk
+constexpr int kPackChunk = 32 * kPackVecs;      // vectors per chunk (1024 bf16 columns)
+
+__global__ void __launch_bounds__(256) ep_pack_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_ids,
+                                                      const float* __restrict__ topk_weights, int64_t T, int H, int topk,
+                                                      int E_rank, int W, const int32_t* __restrict__ row_of,
+                                                      uint16_t* __restrict__ send_x, int32_t* __restrict__ send_ids,
+                                                      float* __restrict__ send_w) {
+  const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t i = warp0; i < rows; i += nwarps) {
-    const int64_t f = send_rows[i];
-    if (f < 0 || f >= T * W) continue;
-    const int64_t t = f / W;
-    const int d = int(f - t * W);
-    if (lane == 0) row_of[f] = int32_t(i);
-    for (int j = lane; j < topk; j += 32) {
-      const int e = __ldg(topk_ids + t * topk + j);
-      const bool here = e >= d * E_rank && e < (d + 1) * E_rank;
-      send_ids[i * topk + j] = here ? e - d * E_rank : -1;
-      send_w[i * topk + j] = here ? __ldg(topk_weights + t * topk + j) : 0.f;
-    }
+  const int64_t cap = T * W;
+  const int nvec = H / 8;
+  const int nchunk = (nvec + kPackChunk - 1) / kPackChunk;
+  for (int64_t unit = warp0; unit < T * nchunk; unit += nwarps) {
+    const int64_t t = unit / nchunk;
+    const int chunk = int(unit - t * nchunk);
+    int i0 = lane < W ? __ldg(row_of + t * W + lane) : -1;
+    int i1 = lane + 32 < W ? __ldg(row_of + t * W + lane + 32) : -1;
+    if (i0 >= cap) i0 = -1;
+    if (i1 >= cap) i1 = -1;
+    const uint32_t m0 = __ballot_sync(0xffffffffu, i0 >= 0), m1 = __ballot_sync(0xffffffffu, i1 >= 0);
+    if ((m0 | m1) == 0) continue;
+    const int v0 = chunk * kPackChunk + lane;
+    uint4 val[kPackVecs];
     const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
-    uint4* dst = reinterpret_cast<uint4*>(send_x + i * H);
-    for (int v = lane; v < H / 8; v += 32) dst[v] = __ldg(src + v);
+#pragma unroll
+    for (int u = 0; u < kPackVecs; ++u)
+      if (v0 + 32 * u < nvec) val[u] = __ldg(src + v0 + 32 * u);
+    for (int h = 0; h < 2; ++h) {
+      uint32_t m = h ? m1 : m0;
+      while (m) {
+        const int dl = __ffs(m) - 1;
+        m &= m - 1;
+        const int d = h * 32 + dl;
+        const int i = __shfl_sync(0xffffffffu, h ? i1 : i0, dl);
+        uint4* dst = reinterpret_cast<uint4*>(send_x + int64_t(i) * H);
+#pragma unroll
+        for (int u = 0; u < kPackVecs; ++u)
+          if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
+        if (chunk == 0) {
+          for (int j = lane; j < topk; j += 32) {
+            const int e = __ldg(topk_ids + t * topk + j);
+            const bool here = e >= d * E_rank && e < (d + 1) * E_rank;
+            send_ids[int64_t(i) * topk + j] = here ? e - d * E_rank : -1;
+            send_w[int64_t(i) * topk + j] = here ? __ldg(topk_weights + t * topk + j) : 0.f;
+          }
+        }
+      }
+    }
   }
 }
 
@@ -131,10 +174,11 @@ cudaError_t launch_ep_pack(const uint16_t* x, const int32_t* topk_ids, const flo
                            int topk, int E_rank, int W, const int32_t* send_rows, const int32_t* rank_offsets,
                            uint16_t* send_x, int32_t* send_ids, float* send_w, int32_t* row_of, int num_sms,
                            cudaStream_t stream) {
-  ep_pack_kernel<<<grid_for(T * W * 32, 256, num_sms), 256, 0, stream>>>(x, topk_ids, topk_weights, T, H, topk, E_rank,
-                                                                         W, send_rows, rank_offsets, send_x, send_ids,
-                                                                         send_w, row_of);
-  count_launches(1);
+  ep_invert_kernel<<<grid_for(T * W, 256, num_sms), 256, 0, stream>>>(send_rows, rank_offsets, T, W, row_of);
+  const int64_t units = T * ((H / 8 + kPackChunk - 1) / kPackChunk);
+  ep_pack_kernel<<<grid_for(units * 32, 256, num_sms), 256, 0, stream>>>(x, topk_ids, topk_weights, T, H, topk, E_rank,
+                                                                         W, row_of, send_x, send_ids, send_w);
+  count_launches(2);
   return cudaGetLastError();
 }
 

@@ -93,8 +93,10 @@ def zipf_popularity(cfg: MoEConfig) -> np.ndarray:
     return p / p.sum()
 
 
-def make_routing(cfg: MoEConfig):
-    """Router output: (topk_ids int32 [T,k] local ids or -1, topk_weights float32 [T,k])."""
+def make_routing(cfg: MoEConfig, global_ids: bool = False):
+    """Router output: (topk_ids int32 [T,k] local ids or -1, topk_weights float32 [T,k]);
+    with global_ids, the ids over all E_global experts (an expert-parallel rank's input
+    to the dispatch)."""
     rng = _streams(cfg.seed)[0]
     T, G, k = cfg.T, cfg.E_global, cfg.topk
     if cfg.routing == "normal":
@@ -113,7 +115,7 @@ def make_routing(cfg: MoEConfig):
     # softmax over all logits then renormalised over the top-k == softmax over the top-k
     z = np.exp(chosen - chosen.max(axis=1, keepdims=True))
     w = (z / z.sum(axis=1, keepdims=True)).astype(np.float32)
-    ids = np.where(sel < cfg.E, sel, -1).astype(np.int32)
+    ids = (sel if global_ids else np.where(sel < cfg.E, sel, -1)).astype(np.int32)
     return np.ascontiguousarray(ids), np.ascontiguousarray(w)
 
 
