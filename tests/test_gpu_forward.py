@@ -132,6 +132,26 @@ def test_ragged_token_counts(chord, T, path):
     assert_layer_close(got, oracle_rows(d, None))
 
 
+# Weight streaming with stream-K (K of at least 512): with fewer (item, stage) units than
+# workers every worker holds about one stage, so an item is split over up to KS workers and
+# its owner adds up to KS - 1 partial sums from other CTAs; mid-size unit counts cut items
+# at arbitrary stages. A second call must give the same bits (the partial sums' flags are
+# reset by the kernel that reads them).
+@pytest.mark.parametrize("T,E,topk,H,I,block_m", [
+    (4, 4, 2, 2048, 256, 8),     # gate_up KS = 4, RU < workers; down K = 256 (short kernel)
+    (5, 3, 3, 3584, 1024, 16),   # KS = 7 and 2, token chunks of 16
+    (16, 8, 2, 7168, 512, 8),    # KS = 14, ranges cut items at any stage
+    (33, 6, 4, 1024, 2048, 32),  # token chunks of 32, down KS = 4
+])
+def test_stream_k_splits_match_the_oracle(chord, T, E, topk, H, I, block_m):
+    d = small_inputs(T, E=E, topk=topk, H=H, I=I, seed=17)
+    layer = make_layer(chord, d, block_m=block_m)
+    first = run_layer(layer, d, chord.CHORD_FLAG_FORCE_STREAM)
+    assert_layer_close(first, oracle_rows(d, None))
+    again = run_layer(layer, d, chord.CHORD_FLAG_FORCE_STREAM)
+    assert np.array_equal(first, again)
+
+
 @pytest.mark.parametrize("path", ["stream", "tensor"])
 def test_no_local_slot_gives_zero_rows(chord, path):
     d = small_inputs(20)
