@@ -150,3 +150,18 @@ def test_ep_send_plan_definition():
     ids = np.array([[0, 5], [6, 7], [-1, 2], [9, 3]], np.int32)   # 2 ranks x 4 experts; 9 is on no rank
     rows, counts = ep_send_plan(ids, 4, 2)
     assert rows == [(0, 0), (2, 0), (3, 0), (0, 1), (1, 1)] and counts == [3, 2]
+
+
+def test_global_ids_restrict_to_the_local_ids():
+    # an expert-parallel rank's router output by global id: its own experts keep their ids,
+    # the others are the ids the layer's local view marks -1
+    sys.path.insert(0, ROOT)
+    from w4a16_int4_mixture_align_b200 import inputs
+    for name in ("ep8_decode", "skew"):
+        cfg = inputs.CONFIGS[name]
+        g, wg = inputs.make_routing(cfg, global_ids=True)
+        loc, wl = inputs.make_routing(cfg)
+        assert g.min() >= 0 and g.max() < cfg.E_global
+        assert np.array_equal(np.where(g < cfg.E, g, -1), loc) and np.array_equal(wg, wl)
+        # every token's top-k experts are distinct
+        assert all(len(set(row)) == cfg.topk for row in g[:64])
