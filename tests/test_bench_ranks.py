@@ -70,3 +70,29 @@ def test_reference_arm_rank0_prints_contract_line():
     assert line["impl"] == "reference" and line["steps"] == 2 and line["unit"] == "us/call"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["higher_is_better"] is False and line["value"] > 0
+
+
+def test_tensor_peak_follows_the_clock_record():
+    # burst cuBLAS figure while the SM clock stays near its maximum; the sustained
+    # (power-capped) figure only when the record shows the clock pulled down by the cap
+    sys.path.insert(0, ROOT)
+    import bench
+    burst, sust = 1642.8, 1402.8
+    assert bench.tensor_peak({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, burst, sust, "m")[0] == burst
+    assert bench.tensor_peak({"sm_mhz": 1916.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}, burst, sust,
+                             "m")[0] == burst
+    assert bench.tensor_peak({"sm_mhz": 1620.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}, burst, sust,
+                             "m")[0] == sust
+    # a low clock with no power-cap reason is not power capping: burst, and the run is
+    # flagged by its clock record instead
+    assert bench.tensor_peak({"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": []}, burst, sust, "m")[0] == burst
+    assert bench.tensor_peak({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}, burst, sust, "m")[0] == burst
+
+
+def test_exchange_workloads_have_no_oracle_arm():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "tp8_reduce"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0
+    import json
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and "unavailable" in line
