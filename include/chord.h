@@ -330,6 +330,17 @@ CHORD_API chord_status_t chord_grouped_masked(const uint16_t* x, int E, int64_t 
  *  chord_moe_forward with CHORD_FLAG_OUTPUT_FP32 writes the rank's FP32 partial output,
  *  the caller all-reduces the partials (sum), and chord_round_bf16 rounds the total once:
  *  out[i] = bf16_rne(in[i]) for i < n (device float in, device bf16 out).
+ *  chord_tp_reduce_round does the all-reduce and the rounding in one pass over the ranks'
+ *  buffers by pointer (peer memory mapped into this process, e.g. over NVLink; or W
+ *  buffers of one GPU standing in for the ranks): rank `rank` of W takes the slice of
+ *  4-float vectors [rank*n/4/W, (rank+1)*n/4/W) and writes outs[d][i] = bf16_rne(
+ *  partials[0][i] + partials[1][i] + ... + partials[W-1][i]) (FP32 sums in rank order, so
+ *  every output holds the same bits) into every rank d's output. partials: W device
+ *  pointers to float [n] (16-byte aligned), outs: W device pointers to bf16 [n] (8-byte
+ *  aligned); both pointer arrays are host memory, read during the call. n % 4 == 0,
+ *  1 <= W <= 64. The caller orders the ranks: every partial is complete before any
+ *  rank's call runs, and an output is complete once every rank's call has run (a barrier
+ *  on each side).
  * All are asynchronous on `stream`; argument errors return before anything is enqueued.
  * ---------------------------------------------------------------------------------- */
 CHORD_API size_t chord_ep_plan_workspace_bytes(int64_t T, int W);
@@ -343,6 +354,8 @@ CHORD_API chord_status_t chord_ep_pack(const uint16_t* hidden, const int32_t* to
 CHORD_API chord_status_t chord_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t T, int H, int W,
                                           uint16_t* out, chord_stream_t stream);
 CHORD_API chord_status_t chord_round_bf16(const float* in, int64_t n, uint16_t* out, chord_stream_t stream);
+CHORD_API chord_status_t chord_tp_reduce_round(const float* const* partials, uint16_t* const* outs, int W, int rank,
+                                               int64_t n, chord_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used by the benchmark).

@@ -196,3 +196,24 @@ def test_round_bf16_matches_the_oracle(chord):
     chord.chord_round_bf16(_dev(v), out)
     torch.cuda.synchronize()
     assert np.array_equal(_bits(out), oracle.f32_to_bf16(v))
+
+
+@pytest.mark.parametrize("W,n", [(4, 4096 * 64), (8, 7168 * 33), (3, 4 * 5), (1, 7168)])
+def test_tp_reduce_round_over_rank_buffers(chord, W, n):
+    # W ranks' buffers on one GPU stand in for peer memory: each rank's call reduces its
+    # slice of all partials in rank order and writes every rank's output; after all W
+    # calls every output is bf16 of the rank-ordered FP32 sum, bit for bit
+    import torch
+    rng = np.random.default_rng(W * 1000 + n % 997)
+    parts = [(rng.standard_normal(n) * 10.0 ** rng.integers(-3, 4, n)).astype(np.float32) for _ in range(W)]
+    ref = parts[0].copy()
+    for p_ in parts[1:]:
+        ref = (ref + p_).astype(np.float32)   # FP32 sums in rank order
+    exp = oracle.f32_to_bf16(ref)
+    d_parts = [_dev(p_) for p_ in parts]
+    outs = [torch.full((n,), 7, dtype=torch.int16, device="cuda").view(torch.bfloat16) for _ in range(W)]
+    for r in range(W):
+        chord.chord_tp_reduce_round(d_parts, outs, r)
+    torch.cuda.synchronize()
+    for o in outs:
+        assert np.array_equal(_bits(o), exp)

@@ -73,6 +73,7 @@ SIGNATURES = {
     "chord_ep_pack": (_I, [_P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "chord_ep_combine": (_I, [_P, _P, _I64, _I, _I, _P, _P]),
     "chord_round_bf16": (_I, [_P, _I64, _P, _P]),
+    "chord_tp_reduce_round": (_I, [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), _I, _I, _I64, _P]),
     "chord_set_timing_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "chord_launch_count": (ctypes.c_uint64, []),
     "chord_selftest_wait_timeout": (_I, [_P, _P, ctypes.c_uint32, _P]),
@@ -271,6 +272,18 @@ def chord_ep_combine(back, row_of, W, out, stream=None):
 def chord_round_bf16(x_f32, out_bf16, stream=None):
     assert x_f32.dtype == torch.float32 and x_f32.numel() == out_bf16.numel()
     _check(lib().chord_round_bf16(_ptr(x_f32), x_f32.numel(), _ptr(out_bf16), _stream(stream)), "chord_round_bf16")
+
+
+def chord_tp_reduce_round(partials, outs, rank, stream=None):
+    """Rank `rank`'s slice of the tensor-parallel all-reduce of the FP32 `partials` (one
+    tensor per rank, readable from this device), rounded to BF16 and stored into every
+    rank's tensor in `outs`."""
+    W = len(partials)
+    assert W == len(outs) and all(p.dtype == torch.float32 and p.numel() == partials[0].numel() for p in partials)
+    assert all(o.numel() == partials[0].numel() for o in outs)
+    ins = (ctypes.c_void_p * W)(*[p.data_ptr() for p in partials])
+    ous = (ctypes.c_void_p * W)(*[o.data_ptr() for o in outs])
+    _check(lib().chord_tp_reduce_round(ins, ous, W, rank, partials[0].numel(), _stream(stream)), "chord_tp_reduce_round")
 
 
 def chord_moe_check_status(workspace, stream=None) -> int:

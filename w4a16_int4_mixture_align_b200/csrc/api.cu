@@ -581,6 +581,29 @@ chord_status_t chord_round_bf16(const float* in, int64_t n, uint16_t* out, chord
   return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "round launch");
 }
 
+chord_status_t chord_tp_reduce_round(const float* const* partials, uint16_t* const* outs, int W, int rank, int64_t n,
+                                    chord_stream_t stream) {
+  clear_detail();
+  if (W < 1 || W > kMaxTpRanks || rank < 0 || rank >= W)
+    return fail(CHORD_ERR_INVALID_ARG, "W=%d rank=%d (1 <= W <= %d)", W, rank, kMaxTpRanks);
+  if (n < 0 || n % 4) return fail(CHORD_ERR_INVALID_ARG, "n=%lld must be a non-negative multiple of 4", (long long)n);
+  if (!partials || !outs) return fail(CHORD_ERR_INVALID_ARG, "null pointer array");
+  TpPeers peers{};
+  for (int s = 0; s < W; ++s) {
+    if (!partials[s] || !outs[s]) return fail(CHORD_ERR_INVALID_ARG, "null pointer for rank %d", s);
+    if ((reinterpret_cast<uintptr_t>(partials[s]) & 15) || (reinterpret_cast<uintptr_t>(outs[s]) & 7))
+      return fail(CHORD_ERR_INVALID_ARG, "rank %d: partials must be 16-byte and outputs 8-byte aligned", s);
+    peers.in[s] = partials[s];
+    peers.out[s] = outs[s];
+  }
+  if (n == 0) return CHORD_OK;
+  chord_status_t st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != CHORD_OK) return st;
+  const cudaError_t err = launch_tp_reduce_round(peers, W, rank, n, num_sms, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? CHORD_OK : cuda_fail(err, "tp reduce launch");
+}
+
 chord_status_t chord_set_timing_events(void* const* events, int n) {
   clear_detail();
   if (n == 0) {

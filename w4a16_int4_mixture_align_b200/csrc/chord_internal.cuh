@@ -471,6 +471,13 @@ cudaError_t launch_ep_pack(const uint16_t* x, const int32_t* topk_ids, const flo
 cudaError_t launch_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t rows_cap, int64_t T, int H, int W,
                               uint16_t* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_round_bf16(const float* in, int64_t n, uint16_t* out, int num_sms, cudaStream_t stream);
+// The ranks' FP32 partials and BF16 outputs of the tensor-parallel reduction, by pointer.
+constexpr int kMaxTpRanks = 64;
+struct TpPeers {
+  const float* in[kMaxTpRanks];
+  uint16_t* out[kMaxTpRanks];
+};
+cudaError_t launch_tp_reduce_round(const TpPeers& peers, int W, int rank, int64_t n, int num_sms, cudaStream_t stream);
 
 // Adds n to the process-wide kernel launch counter (chord_launch_count).
 void count_launches(int n);

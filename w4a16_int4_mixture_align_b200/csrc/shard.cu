@@ -154,6 +154,29 @@ __global__ void __launch_bounds__(256) round_bf16_kernel(const float* __restrict
     out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(in[i]));
 }
 
+// Tensor-parallel reduction over the ranks' buffers by pointer (peer memory, or one GPU's
+// own buffers standing in for the ranks): this rank's slice [v0, v1) of the 4-float
+// vectors, out[d][i] = bf16( sum over s = 0 .. W-1, ascending, of partials[s][i] ) stored
+// into every rank d's output. Every rank sums in the same order, so all outputs agree bit
+// for bit.
+__global__ void __launch_bounds__(256) tp_reduce_round_kernel(TpPeers peers, int W, int64_t v0, int64_t v1) {
+  for (int64_t v = v0 + int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < v1; v += int64_t(gridDim.x) * blockDim.x) {
+    float4 acc = __ldcg(reinterpret_cast<const float4*>(peers.in[0]) + v);
+    for (int s = 1; s < W; ++s) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(peers.in[s]) + v);
+      acc.x = __fadd_rn(acc.x, x.x);
+      acc.y = __fadd_rn(acc.y, x.y);
+      acc.z = __fadd_rn(acc.z, x.z);
+      acc.w = __fadd_rn(acc.w, x.w);
+    }
+    const uint2 o = make_uint2(uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x))) |
+                                   (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16),
+                               uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z))) |
+                                   (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16));
+    for (int d = 0; d < W; ++d) reinterpret_cast<uint2*>(peers.out[d])[v] = o;
+  }
+}
+
 unsigned grid_for(int64_t n, int threads, int num_sms) {
   int64_t g = (n + threads - 1) / threads;
   const int64_t cap = int64_t(num_sms) * 16;
@@ -185,6 +208,15 @@ cudaError_t launch_ep_pack(const uint16_t* x, const int32_t* topk_ids, const flo
 cudaError_t launch_ep_combine(const uint16_t* back, const int32_t* row_of, int64_t rows_cap, int64_t T, int H, int W,
                               uint16_t* out, int num_sms, cudaStream_t stream) {
   ep_combine_kernel<<<grid_for(T * (H / 8), 256, num_sms), 256, 0, stream>>>(back, row_of, rows_cap, T, H, W, out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tp_reduce_round(const TpPeers& peers, int W, int rank, int64_t n, int num_sms, cudaStream_t stream) {
+  const int64_t nv = n / 4;
+  const int64_t v0 = nv * rank / W, v1 = nv * (rank + 1) / W;
+  if (v1 <= v0) return cudaSuccess;
+  tp_reduce_round_kernel<<<grid_for(v1 - v0, 256, num_sms), 256, 0, stream>>>(peers, W, v0, v1);
   count_launches(1);
   return cudaGetLastError();
 }
