@@ -29,8 +29,9 @@ chord_grouped_contiguous / chord_grouped_masked call: routing pass + GEMM) on an
 The exchange workloads time the device steps around a sharded layer on one GPU (the
 collectives between them need several): ep8_exchange_decode / _prefill = chord_ep_plan +
 chord_ep_pack + chord_ep_combine for the EP8 decode (128 tokens) or prefill (8192 tokens)
-batch of one rank over 8 ranks (the returned rows synthetic), and tp8_reduce =
-chord_round_bf16 of the TP8 prefill partial sums.
+batch of one rank over 8 ranks (the returned rows synthetic), tp8_reduce =
+chord_round_bf16 of the TP8 prefill partial sums, and tp8_reduce_peers = the all-reduce
+and rounding by chord_tp_reduce_round over 8 rank buffers of one GPU (all 8 ranks' calls).
 
 --impl reference times the CPU oracle (test infrastructure) on the headline workload on
 the host cores: rank 0 only, other ranks exit without work.
@@ -62,7 +63,7 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 EV_EVERY = 8  # steps per step that records the per-kernel timing events
 DEFAULT_STEPS = {"ep8_decode": 2000, "tp8_decode": 2000, "tiny": 2000, "ep8_prefill": 200,
                  "tp8_prefill": 400, "skew": 100}
-EXCHANGE_WORKLOADS = ("ep8_exchange_decode", "ep8_exchange_prefill", "tp8_reduce")
+EXCHANGE_WORKLOADS = ("ep8_exchange_decode", "ep8_exchange_prefill", "tp8_reduce", "tp8_reduce_peers")
 
 
 def describe(cfg: inputs.MoEConfig) -> str:
@@ -870,6 +871,24 @@ def run_exchange(args, rank, world, local_rank):
                   n_send * H * 2 + T * Wr * 4 + T * H * 2]
         desc = (f"{args.workload}: EP8 batch T={T} top-{k} (global ids) over {Wr} ranks x {E_rank} experts, "
                 f"H={H}: {n_send} send rows; plan + pack + combine (the all-to-all legs not included)")
+    elif args.workload == "tp8_reduce_peers":
+        # 8 ranks' FP32 partials and BF16 outputs as buffers of this GPU; one step runs every
+        # rank's call (its slice reduced in rank order and stored into all 8 outputs): the
+        # whole all-reduce of one TP8 prefill output, emulated on one GPU
+        cfg = inputs.CONFIGS["tp8_prefill"]
+        T, H, Wr = cfg.T, cfg.H, 8
+        rng = np.random.default_rng(rank)
+        host_in = [torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)) for _ in range(Wr)]
+        out_shape, out_dtype = (T, H), torch.bfloat16
+        peer_outs = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(Wr - 1)]
+
+        def steps(xin, oo):
+            outs = [oo] + peer_outs
+            return [lambda r=r: chord.chord_tp_reduce_round(list(xin), outs, r) for r in range(Wr)]
+        names = [f"rank{r}" for r in range(Wr)]
+        nbytes = [Wr * (T * H // Wr) * 4 + Wr * (T * H // Wr) * 2] * Wr
+        desc = (f"tp8_reduce_peers: chord_tp_reduce_round over {Wr} rank buffers of one GPU, FP32 [{T}, {H}] each "
+                f"-> BF16 into all {Wr} outputs (one step = every rank's call)")
     else:
         cfg = inputs.CONFIGS["tp8_prefill"]
         T, H = cfg.T, cfg.H
