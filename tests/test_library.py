@@ -158,3 +158,22 @@ def test_align_size_checks_do_not_overflow(lib):
     f = ctypes.c_void_p(0x100000)
     st = _raw(lib).chord_moe_align(f, (1 << 62) + 1, 64, 48, 8, f, f, f, None, f, 1 << 40, None)
     assert st == lib.CHORD_ERR_UNSUPPORTED and "2^31" in lib.chord_last_error_detail()
+
+
+def test_tp_reduce_round_checks_its_arguments_before_touching_memory(lib):
+    # every rejection happens on the host, before any device access
+    raw = _raw(lib)
+    P = ctypes.c_void_p
+    good_in = (P * 2)(0x100000, 0x200000)
+    good_out = (P * 2)(0x300000, 0x400000)
+    st = raw.chord_tp_reduce_round(good_in, good_out, 0, 0, 64, None)           # W = 0
+    assert st == lib.CHORD_ERR_INVALID_ARG and "W=0" in lib.chord_last_error_detail()
+    assert raw.chord_tp_reduce_round(good_in, good_out, 2, 2, 64, None) == lib.CHORD_ERR_INVALID_ARG   # rank >= W
+    assert raw.chord_tp_reduce_round(good_in, good_out, 65, 0, 64, None) == lib.CHORD_ERR_INVALID_ARG  # W > 64
+    assert raw.chord_tp_reduce_round(good_in, good_out, 2, 0, 6, None) == lib.CHORD_ERR_INVALID_ARG    # n % 4
+    assert raw.chord_tp_reduce_round(None, good_out, 2, 0, 64, None) == lib.CHORD_ERR_INVALID_ARG
+    assert raw.chord_tp_reduce_round((P * 2)(0x100000, None), good_out, 2, 0, 64, None) == lib.CHORD_ERR_INVALID_ARG
+    st = raw.chord_tp_reduce_round((P * 2)(0x100000, 0x200008), good_out, 2, 0, 64, None)   # 8-byte aligned input
+    assert st == lib.CHORD_ERR_INVALID_ARG and "aligned" in lib.chord_last_error_detail()
+    # nothing to do: returns before looking for a device
+    assert raw.chord_tp_reduce_round(good_in, good_out, 2, 1, 0, None) == lib.CHORD_OK
